@@ -1,0 +1,285 @@
+"""fp64 CPU oracle for dynamic top-k block-sparse causal attention (prefill).
+
+TEST INFRASTRUCTURE. Only the tests, the package's smoke check and the
+benchmark's CPU-baseline leg may import or call this module. It shares no
+code with the CUDA path: it never imports the ``dynamic_block_sparse_02_b200``
+package, and that package never imports it.
+
+What is computed, and where the pages say so:
+
+* Block pooling and block scores. Each bs x bs tile of the attention matrix is
+  decided as a unit (zblog.xzdbk.com/559 "dynamic sparse attention" post,
+  section 硬件友好的稀疏计算实现: 64x64 blocks decided per block; "DeepSeek NSA"
+  article, section 2.1: 32x32 blocks whose activation a light per-block
+  predictor estimates). The pages never define the block estimate; the plain
+  reading used here is score(i, j) = mean(Q block i) . mean(K block j).
+* Selection. Each (query head, query block) keeps forced blocks (a local
+  window ending at the diagonal, plus global sink blocks) and the top-k of the
+  remaining causal key blocks (zblog post, section 基于Top-k选择的局部-全局混合:
+  top-k with a local window plus global tokens; "稀疏注意力 vs Flash Attention
+  v2", section 1: content-aware top-k and hybrid local+global modes). The
+  ranking is taken on fp32 scores, because the "DeepSeek NSA" article, section
+  2.2, keeps the routing decision in FP32; the oracle rounds its fp64 score to
+  fp32 once and ranks on that, ties going to the lower block index.
+* Attention. softmax(Q K^T * scale) V over the kept key blocks only, with the
+  causal mask inside the diagonal block ("稀疏注意力 vs Flash Attention v2",
+  section 1 pseudocode: scores, then the sparsity pattern, then softmax with
+  1/sqrt(d_k), then the product with V). Query head h reads KV head
+  h // (Hq/Hkv) (GQA sharing; zblog post, section on speculative decoding,
+  GQA/MQA remark).
+
+Everything is fp64 except the single fp32 rounding of the scores used for
+ranking. The softmax is the exact two-pass form (row max, then the sum of
+exponentials, then the weights), not an online one.
+
+Readings of points the pages leave open (each repeated in the design notes):
+a row whose kept set is empty has output 0 and log-sum-exp -inf; the pooled
+diagonal block is the plain mean of all its rows (the causal mask inside it
+does not enter the pooling); scores are unscaled (a positive scale cannot change
+the ranking).
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, Optional, Sequence, Tuple
+
+import numpy as np
+
+
+# ---------------------------------------------------------------------------
+# Input widening
+# ---------------------------------------------------------------------------
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Widen bf16 bit patterns (uint16) to float64 exactly."""
+    u32 = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return u32.view(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Step 1: block pooling
+# ---------------------------------------------------------------------------
+
+def pool_blocks(x_bits: np.ndarray, block: int) -> np.ndarray:
+    """Block means of a bf16 tensor [B,H,N,d] -> fp64 [B,H,N/block,d].
+
+    pooled[b,h,i,:] = (1/block) * sum over rows r of block i of x[b,h,r,:].
+    The per-block activation estimate of the "DeepSeek NSA" article, section
+    2.1, read as a plain mean over the block's rows.
+    """
+    B, H, N, d = x_bits.shape
+    if N % block:
+        raise ValueError("N must be a multiple of the block size")
+    nb = N // block
+    out = np.empty((B, H, nb, d), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            x = bf16_to_f64(x_bits[b, h])
+            out[b, h] = x.reshape(nb, block, d).mean(axis=1)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Step 2: block scores
+# ---------------------------------------------------------------------------
+
+def block_scores(qp: np.ndarray, kp: np.ndarray) -> np.ndarray:
+    """Causal block scores s[b,h,i,j] = qp[b,h,i] . kp[b, h // g, j] for j <= i.
+
+    Entries above the diagonal (j > i) are -inf. No 1/sqrt(d) factor: a
+    positive scale does not change the ranking ("DeepSeek NSA" section 2.2
+    computes the routing scores at full precision before block sparsifying).
+    """
+    B, Hq, nb, d = qp.shape
+    Hkv = kp.shape[1]
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    g = Hq // Hkv
+    s = np.empty((B, Hq, nb, nb), dtype=np.float64)
+    upper = np.triu(np.ones((nb, nb), dtype=bool), k=1)
+    for b in range(B):
+        for h in range(Hq):
+            s[b, h] = qp[b, h] @ kp[b, h // g].T
+            s[b, h][upper] = -np.inf
+    return s
+
+
+# ---------------------------------------------------------------------------
+# Step 3: selection
+# ---------------------------------------------------------------------------
+
+def forced_set(i: int, local_window: int, n_sink: int) -> set:
+    """Forced key blocks of query block i: the local window {i-w+1 .. i} and sinks {0 .. n_sink-1}.
+
+    zblog post, section 基于Top-k选择的局部-全局混合 (local window plus global
+    tokens); only causal blocks (j <= i) are ever forced.
+    """
+    win = set(range(max(0, i - local_window + 1), i + 1)) if local_window > 0 else set()
+    sink = set(range(0, min(n_sink, i + 1)))
+    return win | sink
+
+
+def row_width(nb: int, k_max: int, local_window: int, n_sink: int) -> int:
+    """Width of one row of the index output: min(nb, k + window + sinks)."""
+    return min(nb, k_max + local_window + n_sink)
+
+
+def select_blocks(scores: np.ndarray, k_free, local_window: int, n_sink: int,
+                  width: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Kept key blocks per (b, query head, query block).
+
+    S(i) = F(i) united with the min(k, |C(i)|) best blocks of
+    C(i) = {0..i} minus F(i), where "best" orders by fp32 score descending, then
+    block index ascending. ``k_free`` is an int, or one int per query head.
+    Returns idx int32 [B,Hq,nb,width] (ascending, padded with -1) and cnt int32
+    [B,Hq,nb].
+    """
+    B, Hq, nb, _ = scores.shape
+    ks = np.full(Hq, int(k_free), dtype=np.int64) if np.isscalar(k_free) else \
+        np.asarray(k_free, dtype=np.int64)
+    if width is None:
+        width = row_width(nb, int(ks.max()) if Hq else 0, local_window, n_sink)
+    idx = np.full((B, Hq, nb, width), -1, dtype=np.int32)
+    cnt = np.zeros((B, Hq, nb), dtype=np.int32)
+    s32 = scores.astype(np.float32)  # the ranking precision (fp32 routing)
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(nb):
+                forced = forced_set(i, local_window, n_sink)
+                free = np.ones(i + 1, dtype=bool)
+                free[sorted(forced)] = False
+                cand = np.nonzero(free)[0].astype(np.int64)
+                take = min(int(ks[h]), cand.size)
+                if take > 0:
+                    # lexsort: last key is primary -> score descending, index ascending
+                    order = np.lexsort((cand, -s32[b, h, i, cand].astype(np.float64)))
+                    picks = cand[order[:take]]
+                else:
+                    picks = np.empty(0, dtype=np.int64)
+                kept = sorted(forced | set(int(j) for j in picks))
+                if len(kept) > width:
+                    raise ValueError("row width too small for the kept set")
+                idx[b, h, i, :len(kept)] = kept
+                cnt[b, h, i] = len(kept)
+    return idx, cnt
+
+
+# ---------------------------------------------------------------------------
+# Step 4: attention over the kept blocks
+# ---------------------------------------------------------------------------
+
+def kept_keys(idx_row: np.ndarray, n: int, block: int) -> np.ndarray:
+    """Token indices of the kept key blocks, ascending."""
+    blocks = np.asarray(idx_row[:n], dtype=np.int64)
+    if blocks.size == 0:
+        return np.empty(0, dtype=np.int64)
+    return (blocks[:, None] * block + np.arange(block)[None, :]).reshape(-1)
+
+
+def block_weights(qblk: np.ndarray, kfull: np.ndarray, keys: np.ndarray, i: int, block: int,
+                  scale: float) -> Tuple[np.ndarray, np.ndarray]:
+    """Exact softmax weights of one query block over the given keys.
+
+    qblk: fp64 [block, d] (rows i*block .. i*block+block-1); kfull: fp64 [N, d].
+    Returns W [block, len(keys)] with zeros at causally masked positions, and
+    lse [block] (natural log; -inf for a row with no visible key).
+    Two passes: row max of the visible logits, then the sum of exponentials.
+    """
+    rows = i * block + np.arange(block)
+    if keys.size == 0:
+        return np.zeros((block, 0)), np.full(block, -np.inf)
+    logits = (qblk @ kfull[keys].T) * scale
+    visible = keys[None, :] <= rows[:, None]
+    logits = np.where(visible, logits, -np.inf)
+    m = logits.max(axis=1)
+    has = np.isfinite(m)
+    m_safe = np.where(has, m, 0.0)
+    e = np.where(visible, np.exp(logits - m_safe[:, None]), 0.0)
+    l = e.sum(axis=1)
+    w = np.where(has[:, None], e / np.where(has, l, 1.0)[:, None], 0.0)
+    lse = np.where(has, m_safe + np.log(np.where(has, l, 1.0)), -np.inf)
+    return w, lse
+
+
+def sparse_attention(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray,
+                     idx: np.ndarray, cnt: np.ndarray, block: int, scale: float = 0.0,
+                     items: Optional[Iterable[Tuple[int, int, int]]] = None):
+    """Block-sparse causal attention over the kept blocks, in fp64.
+
+    O[b,h,r] = sum over visible kept keys t of softmax_t(q_r . k_t * scale) v_t,
+    with K/V of KV head h // (Hq/Hkv). ``scale`` 0 means 1/sqrt(d).
+
+    With ``items`` None, returns (O fp64 [B,Hq,N,d], lse fp64 [B,Hq,N]).
+    Otherwise ``items`` lists (b, h, i) query blocks and the result is a dict
+    mapping each item to (O [block,d], lse [block]).
+    """
+    B, Hq, N, d = q_bits.shape
+    Hkv = k_bits.shape[1]
+    g = Hq // Hkv
+    if scale == 0.0:
+        scale = 1.0 / math.sqrt(d)
+    nb = N // block
+    full = items is None
+    if full:
+        items = [(b, h, i) for b in range(B) for h in range(Hq) for i in range(nb)]
+        out = np.zeros((B, Hq, N, d))
+        lse = np.full((B, Hq, N), -np.inf)
+    else:
+        res = {}
+    items = sorted(items)
+    cache_kv = {}
+    cache_q = {}
+    for (b, h, i) in items:
+        kvh = h // g
+        if (b, kvh) not in cache_kv:
+            cache_kv.clear()
+            cache_kv[(b, kvh)] = (bf16_to_f64(k_bits[b, kvh]), bf16_to_f64(v_bits[b, kvh]))
+        kf, vf = cache_kv[(b, kvh)]
+        if (b, h) not in cache_q:
+            cache_q.clear()
+            cache_q[(b, h)] = bf16_to_f64(q_bits[b, h])
+        qf = cache_q[(b, h)]
+        keys = kept_keys(idx[b, h, i], int(cnt[b, h, i]), block)
+        w, l = block_weights(qf[i * block:(i + 1) * block], kf, keys, i, block, scale)
+        o = w @ vf[keys] if keys.size else np.zeros((block, d))
+        if full:
+            out[b, h, i * block:(i + 1) * block] = o
+            lse[b, h, i * block:(i + 1) * block] = l
+        else:
+            res[(b, h, i)] = (o, l)
+    return (out, lse) if full else res
+
+
+# ---------------------------------------------------------------------------
+# The whole path
+# ---------------------------------------------------------------------------
+
+def forward(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, block: int, k_free,
+            local_window: int, n_sink: int, scale: float = 0.0,
+            items: Optional[Sequence[Tuple[int, int, int]]] = None):
+    """Pool, score, select, attend. Returns (idx, cnt, attention result).
+
+    The attention result is as for ``sparse_attention`` (full arrays, or a dict
+    over ``items``).
+    """
+    qp = pool_blocks(q_bits, block)
+    kp = pool_blocks(k_bits, block)
+    s = block_scores(qp, kp)
+    idx, cnt = select_blocks(s, k_free, local_window, n_sink)
+    att = sparse_attention(q_bits, k_bits, v_bits, idx, cnt, block, scale, items)
+    return idx, cnt, att
+
+
+def attended_pairs(idx: np.ndarray, cnt: np.ndarray, block: int) -> int:
+    """Number of (query, key) score pairs that the kept blocks make visible (causal)."""
+    total = 0
+    for i_flat in np.ndindex(cnt.shape):
+        i = i_flat[-1]
+        for j in idx[i_flat][:cnt[i_flat]]:
+            total += block * (block + 1) // 2 if j == i else block * block
+    return total
+
+
+def dense_pairs(n: int, causal: bool = False) -> int:
+    """Score pairs of dense attention over n tokens: n^2, or n(n+1)/2 with the causal mask."""
+    return n * (n + 1) // 2 if causal else n * n
