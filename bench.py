@@ -1,0 +1,451 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse attention prefill path on B200.
+
+One step = one pass of the whole path over the 32K workload (B=1, 32 query /
+8 KV heads, d=128, 32768 tokens, 64x64 blocks, 64 free picks + 2-block
+window + 1 sink): pool and score the blocks, select them, attend over the
+kept blocks. The step calls dsa_select_blocks then dsa_sparse_attn_fwd, which
+issue the same three kernels as dsa_forward, so that the attention kernel's
+own duration can be read with CUDA events inside the timed region.
+
+Prints ONE JSON line (rank 0). ``--impl reference`` times the fp64 CPU oracle
+instead, on bounded samples of the same workload.
+
+Multi-GPU (torchrun): every rank runs its own independent problem of the same
+shape (weak scaling, no data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from dynamic_block_sparse_02_b200 import WORKLOADS  # noqa: E402
+from dynamic_block_sparse_02_b200 import workloads as W  # noqa: E402
+
+METRIC = "sparse-attn prefill tokens/s at 32K; effective TFLOP/s vs bf16 tensor peak"
+DEFAULT_WORKLOAD = "32k-gqa"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ATTN_SOURCES = ("attn_tc.cu", "attn_mma.cu")
+
+
+# ---------------------------------------------------------------------------
+# host-side helpers (also used by the multi-process CPU tests)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own independent problem."""
+    return 1000 + rank
+
+
+def reduce_max(x: float, device=None) -> float:
+    """Max of a scalar over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(tokens_per_rank_step: int, world: int, steps: int, max_ms: float) -> float:
+    return tokens_per_rank_step * world * steps / (max_ms / 1e3)
+
+
+def kept_flops(cnt_sum: int, block: int, d: int) -> float:
+    """Algorithmic FLOPs of the attention step: 4 * bs^2 * d per kept block
+    (Q K^T and P V, full tiles, diagonal tile counted in full)."""
+    return 4.0 * block * block * d * cnt_sum
+
+
+def select_bytes(w) -> float:
+    """Algorithmic HBM bytes of steps 1-3: Q and K read once, pooled blocks
+    written and read once, index rows and counts written."""
+    q = w.B * w.Hq * w.N * w.d * 2
+    k = w.B * w.Hkv * w.N * w.d * 2
+    pooled = (w.B * w.Hq + w.B * w.Hkv) * w.nb * w.d * 4
+    width = min(w.nb, w.k_free + w.local_window + w.n_sink)
+    sel = w.B * w.Hq * w.nb * (width + 1) * 4
+    return q + k + 2 * pooled + sel
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attn_source_sha() -> str:
+    h = hashlib.sha256()
+    for name in ATTN_SOURCES:
+        p = os.path.join(ROOT, "dynamic_block_sparse_02_b200", "csrc", name)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, or None
+    when the attention kernel's source has changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("source_sha") != attn_source_sha() or rec.get("workload") != workload:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self._t is not None:
+            self._t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample of the workload
+# ---------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(w, x, kph, budget_s: float, seed: int = 0):
+    """Time the oracle on a bounded sample; return (estimated s per full step, description).
+
+    Sample: pooling of all of K plus the pooled Q, scores and selection of the
+    query heads of one KV group; then attention over query blocks of those
+    heads in a seeded random order until ``budget_s`` seconds have passed.
+    The full-step estimate scales selection by Hq / group and attention by
+    (kept blocks of the workload) / (kept blocks processed).
+    """
+    import oracle
+    g = w.group
+    t0 = time.perf_counter()
+    kp = oracle.pool_blocks(x["k"][:, :1], w.block)
+    qp = oracle.pool_blocks(x["q"][:, :g], w.block)
+    s = oracle.block_scores(qp, kp)
+    k = kph[:g] if kph is not None else w.k_free
+    idx, cnt = oracle.select_blocks(s, k, w.local_window, w.n_sink,
+                                    width=min(w.nb, (max(kph) if kph is not None else w.k_free)
+                                              + w.local_window + w.n_sink))
+    t_sel = time.perf_counter() - t0
+    # pooling of Q and K for the remaining heads is part of the full step too
+    t_sel_full = t_sel * (w.Hq / g)
+    rng = np.random.default_rng(seed)
+    order = [(0, h, i) for h in range(g) for i in range(w.nb)]
+    rng.shuffle(order)
+    done, blocks = 0, 0
+    t1 = time.perf_counter()
+    while done < len(order) and time.perf_counter() - t1 < budget_s:
+        chunk = order[done:done + 8]
+        oracle.sparse_attention(x["q"][:, :g], x["k"][:, :1], x["v"][:, :1], idx, cnt, w.block,
+                                items=chunk)
+        blocks += int(sum(cnt[b, h, i] for (b, h, i) in chunk))
+        done += len(chunk)
+    t_att = time.perf_counter() - t1
+    total_blocks = float(cnt.sum()) * (w.B * w.Hq / g)
+    est = t_sel_full + t_att * total_blocks / max(blocks, 1)
+    desc = (f"{w.name}: pooling/scores/selection of {g} query heads (one KV group) timed in full "
+            f"and scaled x{w.Hq // g}; attention on {done} seeded random query blocks "
+            f"({blocks} kept key blocks) timed and scaled to all {int(total_blocks)} kept blocks")
+    return est, desc, t_sel + t_att
+
+
+def run_reference(args, w):
+    """The --impl reference arm: the oracle as it stands, on host cores."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    kph = W.per_head_k(w)
+    kph = None if kph is None else [int(t) for t in kph]
+    x = W.make_inputs(w, seed=rank_seed(0))
+    for _ in range(args.warmup):
+        oracle_sample(w, x, kph, budget_s=1.0)
+    ests, desc = [], ""
+    for s in range(args.steps):
+        est, desc, _ = oracle_sample(w, x, kph, budget_s=args.ref_budget, seed=s)
+        ests.append(est)
+    est = statistics.median(ests)
+    tokens = w.B * w.N
+    value = tokens / est
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+            "block": w.block, "k_free": w.k_free, "local_window": w.local_window,
+            "n_sink": w.n_sink,
+            "l2": "inputs larger than L2: Q+K+V = %.0f MB per step > 126 MB"
+                  % ((w.B * (w.Hq + 2 * w.Hkv) * w.N * w.d * 2) / 1e6)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+    from dynamic_block_sparse_02_b200 import binding as B
+    from dynamic_block_sparse_02_b200.attention import BlockSparseAttention
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    kph = W.per_head_k(w)
+    kph = None if kph is None else [int(t) for t in kph]
+    x = W.make_inputs(w, seed=rank_seed(rank))
+    to_t = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    q_h, k_h, v_h = (to_t(x[n]).pin_memory() for n in ("q", "k", "v"))
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    stream = torch.cuda.Stream(device=dev)
+    att = BlockSparseAttention.from_workload(w, k_per_head=kph, device=dev, stream=stream,
+                                             attn_kernel=args.attn_kernel)
+    idx, cnt = att.empty_selection()
+    out = att.empty_out()
+
+    def select():
+        B.dsa_select_blocks(att.params, q, k, idx, cnt, att.ws, att.ws_bytes, stream)
+
+    def attend():
+        B.dsa_sparse_attn_fwd(att.params, q, k, v, idx, cnt, out, None, att.ws, att.ws_bytes, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            select()
+            attend()
+    torch.cuda.synchronize(dev)
+    status = B.dsa_check_status(att.ws, stream)
+    if status != B.DSA_OK:
+        raise RuntimeError("device error during warm-up: " + B.status_string(status))
+    kept = int(cnt.sum().item())
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    if rank == 0 and not args.no_clocks:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for s in range(K):
+            ev[s][0].record(stream)
+            select()
+            ev[s][1].record(stream)
+            attend()
+            ev[s][2].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if rank == 0 else None
+    status = B.dsa_check_status(att.ws, stream)
+    if status != B.DSA_OK:
+        raise RuntimeError("device error during timing: " + B.status_string(status))
+
+    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    sel_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    att_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    max_total = reduce_max(total_ms, dev)
+    tokens = w.B * w.N
+    value = whole_job_tokens_per_s(tokens, world, K, max_total)
+
+    # end to end through the public call, with host buffers and copies inside the timed region
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    Ke = max(3, min(K, args.e2e_steps))
+
+    def e2e_step():
+        q.copy_(q_h, non_blocking=True)
+        k.copy_(k_h, non_blocking=True)
+        v.copy_(v_h, non_blocking=True)
+        att.forward(q, k, v, out)
+        out_h.copy_(out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
+    e2e_value = whole_job_tokens_per_s(tokens, world, Ke, e2e_ms)
+    status = B.dsa_check_status(att.ws, stream)
+    if status != B.DSA_OK:
+        raise RuntimeError("device error in the end-to-end loop: " + B.status_string(status))
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_kind = load_peaks()
+    att_avg = statistics.mean(att_ms)
+    sel_avg = statistics.mean(sel_ms)
+    flops = kept_flops(kept, w.block, w.d)
+    achieved = flops / (att_avg / 1e3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    sel_gbs = select_bytes(w) / (sel_avg / 1e3) / 1e9
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        est, desc, spent = oracle_sample(w, x, kph, budget_s=args.cpu_budget)
+        cpu = {"value": tokens / est, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc + f" ({spent:.1f} s of CPU work)"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": max_total / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(w),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": recorded_traffic(w.name),
+                     "kernel": "sparse attention (dsa_sparse_attn_fwd)",
+                     "peak_kind": f"{peak_kind} bf16 dense, sustained",
+                     "frac_of_burst": achieved / float(peaks["bf16_tflops"])},
+        "select": {"ms": sel_avg, "algorithmic_bytes": select_bytes(w), "GBps": sel_gbs,
+                   "frac_hbm": sel_gbs / float(peaks["hbm_gbs"]), "bound": "hbm"},
+        "attention_ms": att_avg,
+        "kept_blocks_per_step": kept,
+        "effective_tflops": achieved,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": int(q_h.numel() + k_h.numel() + v_h.numel()) * 2,
+                "d2h_bytes_per_step": int(out_h.numel()) * 2},
+        "gpu_launches": 3 * K,
+        "clocks": clocks,
+        "attn_kernel": {0: "auto", 1: "tcgen05", 2: "mma.sync"}[args.attn_kernel],
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--attn-kernel", type=int, default=0, choices=[0, 1, 2])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

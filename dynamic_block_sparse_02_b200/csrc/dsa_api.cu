@@ -1,0 +1,290 @@
+// C-ABI entry points of libdsa (declared in include/dsa.h): argument checks,
+// workspace layout and kernel launches. No entry point allocates memory or
+// synchronises the host, except dsa_check_status, which synchronises on
+// purpose to read the device error flag.
+#include <cmath>
+#include <cstring>
+
+#include "dsa_internal.cuh"
+
+using dsa::Shape;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_empty(const dsa_params* p) { return p->B == 0 || p->N == 0; }
+
+// Checks every field and derives the shape. Empty problems (B or N zero)
+// are valid; their other fields must still be well formed.
+dsa_status make_shape(const dsa_params* p, Shape* s) {
+  if (p == nullptr) return DSA_ERR_INVALID_ARG;
+  if (p->B < 0 || p->N < 0 || p->Hq < 1 || p->Hkv < 1 || p->d < 1 || p->block < 1)
+    return DSA_ERR_INVALID_ARG;
+  if (p->Hq % p->Hkv != 0) return DSA_ERR_INVALID_ARG;
+  if (p->local_window < 0 || p->n_sink < 0) return DSA_ERR_INVALID_ARG;
+  if (!std::isfinite(p->scale) || p->scale < 0.f) return DSA_ERR_INVALID_ARG;
+  if (p->attn_kernel < DSA_ATTN_AUTO || p->attn_kernel > DSA_ATTN_MMA_SYNC)
+    return DSA_ERR_INVALID_ARG;
+  long long kmax_head = 0;
+  if (p->k_per_head != nullptr) {
+    if (p->Hq > dsa::kMaxHeads) return DSA_ERR_UNSUPPORTED;
+    for (int h = 0; h < p->Hq; ++h) {
+      if (p->k_per_head[h] < 0) return DSA_ERR_INVALID_ARG;
+      if (p->k_per_head[h] > kmax_head) kmax_head = p->k_per_head[h];
+    }
+  } else {
+    if (p->k_free < 0) return DSA_ERR_INVALID_ARG;
+    kmax_head = p->k_free;
+  }
+  if (p->d != 64 && p->d != 128) return DSA_ERR_UNSUPPORTED;
+  if (p->block != 32 && p->block != 64 && p->block != 128) return DSA_ERR_UNSUPPORTED;
+  if (p->N % p->block != 0) return DSA_ERR_UNSUPPORTED;
+  const int nb = p->N / p->block;
+  if (nb > dsa::kMaxBlocks) return DSA_ERR_UNSUPPORTED;
+  // element counts must stay well inside 64-bit and the grids inside 2^31
+  const long long elems = (long long)p->B * p->Hq * p->N * p->d;
+  if ((long long)p->B * p->Hq * nb > 0x7fffffffLL || elems > (1LL << 40))
+    return DSA_ERR_UNSUPPORTED;
+  s->B = p->B;
+  s->Hq = p->Hq;
+  s->Hkv = p->Hkv;
+  s->N = p->N;
+  s->d = p->d;
+  s->bs = p->block;
+  s->nb = nb;
+  s->group = p->Hq / p->Hkv;
+  s->lw = p->local_window;
+  s->ns = p->n_sink;
+  long long w = kmax_head + (long long)p->local_window + (long long)p->n_sink;
+  s->W = (int)(w < nb ? w : nb);
+  s->scale = p->scale == 0.f ? 1.0f / std::sqrt((float)p->d) : p->scale;
+  s->kmax_head = (int)(kmax_head < nb ? kmax_head : nb);
+  s->per_head = p->k_per_head != nullptr;
+  return DSA_OK;
+}
+
+struct Layout {
+  size_t qp, kp, idx, cnt, total;
+};
+
+Layout layout(const Shape& s) {
+  Layout L;
+  size_t off = dsa::kHeaderBytes;
+  L.qp = off;
+  off += round_up((size_t)s.B * s.Hq * s.nb * s.d * sizeof(float));
+  L.kp = off;
+  off += round_up((size_t)s.B * s.Hkv * s.nb * s.d * sizeof(float));
+  L.idx = off;
+  off += round_up((size_t)s.B * s.Hq * s.nb * s.W * sizeof(int32_t));
+  L.cnt = off;
+  off += round_up((size_t)s.B * s.Hq * s.nb * sizeof(int32_t));
+  L.total = off;
+  return L;
+}
+
+dsa_status check_ws(const Shape& s, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr || !aligned16(ws)) return DSA_ERR_WORKSPACE;
+  if (ws_bytes < layout(s).total) return DSA_ERR_WORKSPACE;
+  return DSA_OK;
+}
+
+// The device must be Blackwell sm_100; results are cached per device.
+dsa_status check_device() {
+  static int cached[64] = {0};  // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
+  if (dev >= 0 && dev < 64 && cached[dev] != 0) return cached[dev] == 1 ? DSA_OK : DSA_ERR_UNSUPPORTED;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  const bool ok = major == 10 && minor == 0;
+  if (dev >= 0 && dev < 64) cached[dev] = ok ? 1 : 2;
+  return ok ? DSA_OK : DSA_ERR_UNSUPPORTED;
+}
+
+dsa::KBudget budgets(const dsa_params* p) {
+  dsa::KBudget kb;
+  std::memset(&kb, 0, sizeof(kb));
+  if (p->k_per_head != nullptr) {
+    for (int h = 0; h < p->Hq; ++h) kb.k[h] = p->k_per_head[h];
+  } else {
+    kb.k[0] = p->k_free;
+  }
+  return kb;
+}
+
+dsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+dsa_status run_attention(const dsa_params* p, const Shape& s, const dsa_bf16* q, const dsa_bf16* k,
+                         const dsa_bf16* v, const int32_t* idx, const int32_t* cnt, dsa_bf16* out,
+                         float* lse, dsa::WsHeader* hdr, cudaStream_t st) {
+  auto bq = reinterpret_cast<const __nv_bfloat16*>(q);
+  auto bk = reinterpret_cast<const __nv_bfloat16*>(k);
+  auto bv = reinterpret_cast<const __nv_bfloat16*>(v);
+  auto bo = reinterpret_cast<__nv_bfloat16*>(out);
+  const bool tc_ok = dsa::attn_tc_supported(s);
+  if (p->attn_kernel == DSA_ATTN_TCGEN05 && !tc_ok) return DSA_ERR_UNSUPPORTED;
+  if (p->attn_kernel != DSA_ATTN_MMA_SYNC && tc_ok)
+    return from_cuda(dsa::launch_attn_tc(s, bq, bk, bv, idx, cnt, bo, lse, hdr, st));
+  return from_cuda(dsa::launch_attn_mma(s, bq, bk, bv, idx, cnt, bo, lse, hdr, st));
+}
+
+// Steps 1-3: pooling, then the fused score + select kernel.
+dsa_status run_selection(const dsa_params* p, const Shape& s, const dsa_bf16* q, const dsa_bf16* k,
+                         int32_t* idx, int32_t* cnt, void* ws, cudaStream_t st) {
+  const Layout L = layout(s);
+  char* base = static_cast<char*>(ws);
+  auto hdr = reinterpret_cast<dsa::WsHeader*>(base);
+  float* qp = reinterpret_cast<float*>(base + L.qp);
+  float* kp = reinterpret_cast<float*>(base + L.kp);
+  cudaError_t e = dsa::launch_pool(s, reinterpret_cast<const __nv_bfloat16*>(q),
+                                   reinterpret_cast<const __nv_bfloat16*>(k), qp, kp, st);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  return from_cuda(dsa::launch_score_select(s, budgets(p), qp, kp, idx, cnt, hdr, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dsa_kmax(const dsa_params* p) {
+  Shape s;
+  if (make_shape(p, &s) != DSA_OK || is_empty(p)) return 0;
+  return (size_t)s.W;
+}
+
+dsa_status dsa_workspace_size(const dsa_params* p, size_t* bytes) {
+  if (bytes == nullptr) return DSA_ERR_INVALID_ARG;
+  Shape s;
+  dsa_status st = make_shape(p, &s);
+  if (st != DSA_OK) return st;
+  *bytes = is_empty(p) ? dsa::kHeaderBytes : layout(s).total;
+  return DSA_OK;
+}
+
+dsa_status dsa_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < dsa::kHeaderBytes) return DSA_ERR_WORKSPACE;
+  return from_cuda(cudaMemsetAsync(ws, 0, dsa::kHeaderBytes, (cudaStream_t)stream));
+}
+
+dsa_status dsa_block_scores(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k,
+                            float* scores, void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  dsa_status st = make_shape(p, &s);
+  if (st != DSA_OK) return st;
+  if (is_empty(p)) return DSA_OK;
+  if (q == nullptr || k == nullptr || scores == nullptr || !aligned16(q) || !aligned16(k) ||
+      !aligned16(scores))
+    return DSA_ERR_INVALID_ARG;
+  if ((st = check_ws(s, ws, ws_bytes)) != DSA_OK) return st;
+  if ((st = check_device()) != DSA_OK) return st;
+  const Layout L = layout(s);
+  char* base = static_cast<char*>(ws);
+  float* qp = reinterpret_cast<float*>(base + L.qp);
+  float* kp = reinterpret_cast<float*>(base + L.kp);
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = dsa::launch_pool(s, reinterpret_cast<const __nv_bfloat16*>(q),
+                                   reinterpret_cast<const __nv_bfloat16*>(k), qp, kp, cs);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  return from_cuda(dsa::launch_scores(s, qp, kp, scores, cs));
+}
+
+dsa_status dsa_topk_select(const dsa_params* p, const float* scores, int32_t* idx, int32_t* cnt,
+                           void* stream) {
+  Shape s;
+  dsa_status st = make_shape(p, &s);
+  if (st != DSA_OK) return st;
+  if (is_empty(p)) return DSA_OK;
+  if (scores == nullptr || idx == nullptr || cnt == nullptr || !aligned16(scores))
+    return DSA_ERR_INVALID_ARG;
+  if ((st = check_device()) != DSA_OK) return st;
+  return from_cuda(dsa::launch_select(s, budgets(p), scores, idx, cnt, nullptr, (cudaStream_t)stream));
+}
+
+dsa_status dsa_select_blocks(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k,
+                             int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  dsa_status st = make_shape(p, &s);
+  if (st != DSA_OK) return st;
+  if (is_empty(p)) return DSA_OK;
+  if (q == nullptr || k == nullptr || idx == nullptr || cnt == nullptr || !aligned16(q) ||
+      !aligned16(k))
+    return DSA_ERR_INVALID_ARG;
+  if ((st = check_ws(s, ws, ws_bytes)) != DSA_OK) return st;
+  if ((st = check_device()) != DSA_OK) return st;
+  return run_selection(p, s, q, k, idx, cnt, ws, (cudaStream_t)stream);
+}
+
+dsa_status dsa_sparse_attn_fwd(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k,
+                               const dsa_bf16* v, const int32_t* idx, const int32_t* cnt,
+                               dsa_bf16* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  dsa_status st = make_shape(p, &s);
+  if (st != DSA_OK) return st;
+  if (is_empty(p)) return DSA_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || idx == nullptr || cnt == nullptr ||
+      out == nullptr || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return DSA_ERR_INVALID_ARG;
+  if ((st = check_ws(s, ws, ws_bytes)) != DSA_OK) return st;
+  if ((st = check_device()) != DSA_OK) return st;
+  auto hdr = static_cast<dsa::WsHeader*>(ws);
+  return run_attention(p, s, q, k, v, idx, cnt, out, lse, hdr, (cudaStream_t)stream);
+}
+
+dsa_status dsa_forward(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k, const dsa_bf16* v,
+                       dsa_bf16* out, float* lse, int32_t* idx, int32_t* cnt, void* ws,
+                       size_t ws_bytes, void* stream) {
+  Shape s;
+  dsa_status st = make_shape(p, &s);
+  if (st != DSA_OK) return st;
+  if (is_empty(p)) return DSA_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || !aligned16(q) ||
+      !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return DSA_ERR_INVALID_ARG;
+  if ((idx == nullptr) != (cnt == nullptr)) return DSA_ERR_INVALID_ARG;
+  if ((st = check_ws(s, ws, ws_bytes)) != DSA_OK) return st;
+  if ((st = check_device()) != DSA_OK) return st;
+  const Layout L = layout(s);
+  char* base = static_cast<char*>(ws);
+  auto hdr = reinterpret_cast<dsa::WsHeader*>(base);
+  if (idx == nullptr) {
+    idx = reinterpret_cast<int32_t*>(base + L.idx);
+    cnt = reinterpret_cast<int32_t*>(base + L.cnt);
+  }
+  cudaStream_t cs = (cudaStream_t)stream;
+  if ((st = run_selection(p, s, q, k, idx, cnt, ws, cs)) != DSA_OK) return st;
+  return run_attention(p, s, q, k, v, idx, cnt, out, lse, hdr, cs);
+}
+
+dsa_status dsa_check_status(void* ws, void* stream) {
+  if (ws == nullptr || !aligned16(ws)) return DSA_ERR_WORKSPACE;
+  cudaStream_t cs = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return DSA_ERR_CUDA;
+  int flag = 0;
+  if (cudaMemcpy(&flag, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
+  if (flag != 0) {
+    if (cudaMemset(ws, 0, 4 * sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
+  }
+  return (dsa_status)flag;
+}
+
+const char* dsa_status_string(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape or device";
+    case DSA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case DSA_ERR_CUDA: return "CUDA runtime or launch error";
+    case DSA_ERR_DEVICE_TIMEOUT: return "a bounded wait on the device gave up";
+    case DSA_ERR_DEVICE_BOUNDS: return "a kernel met an index out of range";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// Internal declarations shared by the kernels and the C-ABI host code.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "../../include/dsa.h"
+
+namespace dsa {
+
+// Workspace header (the first kHeaderBytes of the caller's workspace).
+struct WsHeader {
+  int status;           // first device-side error (dsa_status value), 0 = none
+  int detail[3];        // kernel id and a coordinate of the first error
+  unsigned int work[8]; // work counters of persistent kernels (reset per call)
+};
+constexpr size_t kHeaderBytes = 256;
+static_assert(sizeof(WsHeader) <= kHeaderBytes, "header too large");
+
+constexpr int kMaxBlocks = 1024;  // largest nb = N / block
+constexpr int kMaxHeads = 256;    // largest Hq when k_per_head is given
+
+// Kernel ids reported in WsHeader::detail[0].
+enum KernelId { kKernPool = 1, kKernScore = 2, kKernSelect = 3, kKernAttnMma = 4, kKernAttnTc = 5 };
+
+// Derived, validated problem description.
+struct Shape {
+  int B, Hq, Hkv, N, d, bs, nb, group, W;
+  int lw, ns;
+  float scale;
+  int kmax_head;
+  bool per_head;
+};
+
+// Per-head top-k budgets passed by value to the kernels.
+struct KBudget {
+  int32_t k[kMaxHeads];
+};
+
+// Device-side error reporting: the first error wins.
+__device__ __forceinline__ void raise_error(WsHeader* hdr, int status, int kernel, int a, int b) {
+  if (hdr == nullptr) return;
+  if (atomicCAS(&hdr->status, 0, status) == 0) {
+    hdr->detail[0] = kernel;
+    hdr->detail[1] = a;
+    hdr->detail[2] = b;
+  }
+}
+
+// Launchers (return cudaSuccess or the launch error).
+cudaError_t launch_pool(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, float* qp,
+                        float* kp, cudaStream_t st);
+cudaError_t launch_scores(const Shape& s, const float* qp, const float* kp, float* scores,
+                          cudaStream_t st);
+cudaError_t launch_score_select(const Shape& s, const KBudget& kb, const float* qp, const float* kp,
+                                int32_t* idx, int32_t* cnt, WsHeader* hdr, cudaStream_t st);
+cudaError_t launch_select(const Shape& s, const KBudget& kb, const float* scores, int32_t* idx,
+                          int32_t* cnt, WsHeader* hdr, cudaStream_t st);
+cudaError_t launch_attn_mma(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                            const __nv_bfloat16* v, const int32_t* idx, const int32_t* cnt,
+                            __nv_bfloat16* out, float* lse, WsHeader* hdr, cudaStream_t st);
+bool attn_tc_supported(const Shape& s);
+cudaError_t launch_attn_tc(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                           const __nv_bfloat16* v, const int32_t* idx, const int32_t* cnt,
+                           __nv_bfloat16* out, float* lse, WsHeader* hdr, cudaStream_t st);
+
+}  // namespace dsa

@@ -1,0 +1,173 @@
+/*
+ * dsa.h — C ABI of libdsa: dynamic top-k block-sparse causal attention
+ * (prefill) on NVIDIA B200 (sm_100a).
+ *
+ * The operation, as the pages describe it:
+ *   1. Pool.   Each bs x bs tile of the attention matrix is decided as a unit
+ *              (zblog.xzdbk.com/559 dynamic-sparse-attention post, section
+ *              硬件友好的稀疏计算实现, 64x64 blocks; "DeepSeek NSA" article,
+ *              section 2.1, 32x32 blocks with a light per-block estimate).
+ *              The estimate used here: Qp[i] = mean of query block i,
+ *              Kp[j] = mean of key block j (fp32).
+ *   2. Score.  s(i, j) = Qp[i] . Kp[j] for j <= i, in fp32 ("DeepSeek NSA",
+ *              section 2.2: the routing decision stays in FP32).
+ *   3. Select. Per (batch, query head, query block i): the forced blocks
+ *              F(i) = {i-w+1 .. i} U {0 .. n_sink-1} (causal part only) plus the
+ *              k best remaining causal blocks, best = higher score, ties to
+ *              the lower block index (zblog post, section
+ *              基于Top-k选择的局部-全局混合: top-k with local window and global
+ *              tokens).
+ *   4. Attend. O = softmax(Q K^T * scale) V over the kept blocks only, causal
+ *              inside the diagonal block, online softmax, query head h reading
+ *              KV head h / (Hq/Hkv) ("稀疏注意力 vs Flash Attention v2",
+ *              section 1 pseudocode; "DeepSeek NSA", section 2.2, bf16 matmul).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are DEVICE pointers to contiguous row-major arrays, d innermost:
+ *     Q and O [B, Hq, N, d]; K and V [B, Hkv, N, d]; all bf16 (dsa_bf16 is the
+ *     16-bit pattern of one bfloat16). Q, K, V, O and the workspace must be
+ *     16-byte aligned.
+ *   - Block index rows: idx int32 [B, Hq, nb, W] with nb = N / block and
+ *     W = dsa_kmax(p); each row lists its kept key blocks in ascending order,
+ *     padded with -1; cnt int32 [B, Hq, nb] holds each row's length.
+ *   - The caller owns all memory. The library never allocates device or host
+ *     memory; it uses the caller's workspace (dsa_workspace_size bytes).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and do not synchronise the host, so a sequence of calls
+ *     can be captured into a CUDA graph.
+ *   - An argument error is reported synchronously by the return value and
+ *     launches nothing. Errors found on the device (an index out of range, a
+ *     bounded wait that gave up) set a flag in the workspace header; read it
+ *     with dsa_check_status.
+ *   - The device must be an sm_100a GPU (B200). The library holds no state
+ *     except, per device, a cache of the kernels' shared-memory attributes.
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t dsa_bf16; /* bit pattern of one bfloat16 value */
+
+typedef enum dsa_status {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,    /* a null/misaligned pointer, a negative size, Hq % Hkv != 0, ... */
+  DSA_ERR_UNSUPPORTED = 2,    /* valid but outside the supported shapes (see dsa_params) */
+  DSA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than dsa_workspace_size */
+  DSA_ERR_CUDA = 4,           /* a CUDA runtime call or a kernel launch failed */
+  DSA_ERR_DEVICE_TIMEOUT = 5, /* a bounded wait inside a kernel gave up (device flag) */
+  DSA_ERR_DEVICE_BOUNDS = 6   /* a kernel met an index outside its valid range (device flag) */
+} dsa_status;
+
+/* Attention kernel choice (dsa_params.attn_kernel). */
+typedef enum dsa_attn_kernel {
+  DSA_ATTN_AUTO = 0,     /* the fastest kernel this library has for the shape */
+  DSA_ATTN_TCGEN05 = 1,  /* tcgen05/TMEM tensor-core kernel with TMA tile loads */
+  DSA_ATTN_MMA_SYNC = 2  /* warp-level mma.sync kernel (the legacy tensor-core path) */
+} dsa_attn_kernel;
+
+/*
+ * Problem shape and selection settings.
+ *   B, Hq, Hkv, N, d : batch, query heads, KV heads, tokens, head dim.
+ *                      Hq % Hkv == 0; d is 64 or 128; B == 0 or N == 0 is an
+ *                      empty problem (every call returns DSA_OK, launches nothing).
+ *   block            : tile edge bs, one of 32, 64, 128; N % block == 0;
+ *                      nb = N / block must be <= 1024.
+ *   k_free           : top-k picks beyond the forced set, for every head
+ *                      (used when k_per_head is NULL); >= 0.
+ *   k_per_head       : optional HOST array of Hq budgets (>= 0), shared across
+ *                      the batch; read during the call only. Hq <= 256 then.
+ *   local_window     : w >= 0; forces blocks {i-w+1 .. i} (1 = diagonal only).
+ *   n_sink           : >= 0; forces blocks {0 .. n_sink-1}.
+ *   scale            : softmax scale; 0 means 1/sqrt(d); must be finite, >= 0.
+ *   attn_kernel      : a dsa_attn_kernel value.
+ */
+typedef struct dsa_params {
+  int B, Hq, Hkv, N, d;
+  int block;
+  int k_free;
+  const int32_t *k_per_head;
+  int local_window;
+  int n_sink;
+  float scale;
+  int attn_kernel;
+} dsa_params;
+
+/* Row width W of idx: min(nb, max_h k_h + local_window + n_sink). 0 for an
+ * invalid or empty problem. */
+size_t dsa_kmax(const dsa_params *p);
+
+/* Bytes of device workspace the calls below need for this problem (*bytes is
+ * set on success). The first 256 bytes are a header (device error flag, work
+ * counters); zero them once after allocating (dsa_workspace_init). */
+dsa_status dsa_workspace_size(const dsa_params *p, size_t *bytes);
+
+/* Zero the workspace header on `stream` (asynchronous). */
+dsa_status dsa_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Steps 1-2. scores: device fp32 [B, Hq, nb, nb]; scores[b,h,i,j] =
+ * Qp[b,h,i] . Kp[b,h/(Hq/Hkv),j] for j <= i and -inf for j > i.
+ * Uses the workspace for the pooled blocks.
+ */
+dsa_status dsa_block_scores(const dsa_params *p, const dsa_bf16 *q, const dsa_bf16 *k,
+                            float *scores, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Step 3 on caller scores laid out as dsa_block_scores writes them (only the
+ * entries j <= i are read). Writes idx [B,Hq,nb,W] and cnt [B,Hq,nb]. Given
+ * the scores of dsa_block_scores, the result equals the selection inside
+ * dsa_forward bit for bit.
+ */
+dsa_status dsa_topk_select(const dsa_params *p, const float *scores, int32_t *idx,
+                           int32_t *cnt, void *stream);
+
+/*
+ * Steps 1-3 in one call (pool, score, select); the scores stay on chip and
+ * only the selection is written: idx [B,Hq,nb,W], cnt [B,Hq,nb]. The result
+ * equals dsa_block_scores followed by dsa_topk_select, bit for bit, and is the
+ * selection dsa_forward uses.
+ */
+dsa_status dsa_select_blocks(const dsa_params *p, const dsa_bf16 *q, const dsa_bf16 *k,
+                             int32_t *idx, int32_t *cnt, void *ws, size_t ws_bytes,
+                             void *stream);
+
+/*
+ * Step 4 on a caller selection. idx/cnt as above, W = dsa_kmax(p); every
+ * entry n < cnt must satisfy 0 <= idx <= i, and a row must be ascending
+ * without repeats (the kernel skips an out-of-range entry and sets
+ * DSA_ERR_DEVICE_BOUNDS; order and repeats are not checked). out: bf16
+ * [B,Hq,N,d] (round to nearest even). lse: optional fp32 [B,Hq,N], natural-log
+ * log-sum-exp of the scaled logits of each row. A row with no visible key
+ * gets out = 0 and lse = -inf.
+ */
+dsa_status dsa_sparse_attn_fwd(const dsa_params *p, const dsa_bf16 *q, const dsa_bf16 *k,
+                               const dsa_bf16 *v, const int32_t *idx, const int32_t *cnt,
+                               dsa_bf16 *out, float *lse, void *ws, size_t ws_bytes,
+                               void *stream);
+
+/*
+ * Steps 1-4 in one call; the scores never reach device memory. idx/cnt are
+ * optional outputs (NULL keeps them in the workspace); lse is optional.
+ */
+dsa_status dsa_forward(const dsa_params *p, const dsa_bf16 *q, const dsa_bf16 *k,
+                       const dsa_bf16 *v, dsa_bf16 *out, float *lse, int32_t *idx,
+                       int32_t *cnt, void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronise `stream`, read the device error flag in the workspace header,
+ * clear it, and return it (DSA_OK if no kernel raised one). */
+dsa_status dsa_check_status(void *ws, void *stream);
+
+/* Static English text for a status value. */
+const char *dsa_status_string(dsa_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

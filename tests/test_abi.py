@@ -1,0 +1,141 @@
+"""The C-ABI boundary on the host: the library loads, exports every declared
+symbol, sizes its outputs and workspace, and rejects bad arguments with the
+documented status before touching the device. No test here launches a kernel.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from dynamic_block_sparse_02_b200 import WORKLOADS, binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+FAKE = 0x10000  # an aligned non-null address; never dereferenced by these tests
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    for n in ("dsa_block_scores", "dsa_topk_select", "dsa_sparse_attn_fwd", "dsa_forward",
+              "dsa_workspace_size", "dsa_kmax", "dsa_check_status", "dsa_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(dsa_\w+)", out))
+    assert set(names) <= exported, set(names) - exported
+    for n in names:
+        assert hasattr(B.raw(n), "__call__")
+    assert set(names) == set(B.SIGNATURES)
+
+
+def test_status_strings():
+    for s in range(7):
+        assert B.status_string(s) and B.status_string(s) != "unknown status"
+    assert B.status_string(99) == "unknown status"
+
+
+def kept_width(w, kmax_head):
+    return min(w.nb, kmax_head + w.local_window + w.n_sink)
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_kmax_and_workspace_size(name):
+    w = WORKLOADS[name]
+    kph = [8, 16, 32, 64] * (w.Hq // 4) if w.k_choices else None
+    p = B.Params.from_workload(w, k_per_head=kph)
+    width = B.dsa_kmax(p)
+    assert width == kept_width(w, 64 if kph else w.k_free)
+    expect = {"tiny": 4, "8k-gqa": 18, "32k-gqa": 67, "128k-structured": 65, "batched-32": 65}[name]
+    assert width == expect
+    ws = B.dsa_workspace_size(p)
+    rnd = lambda x: (x + 255) // 256 * 256
+    expect_ws = 256 + rnd(w.B * w.Hq * w.nb * w.d * 4) + rnd(w.B * w.Hkv * w.nb * w.d * 4) \
+        + rnd(w.B * w.Hq * w.nb * width * 4) + rnd(w.B * w.Hq * w.nb * 4)
+    assert ws == expect_ws
+
+
+def status_of_forward(p, q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=None, idx=None, cnt=None, ws=FAKE,
+                      ws_bytes=1 << 40):
+    return B.raw("dsa_forward")(p.ref, q, k, v, out, lse, idx, cnt, ws, ws_bytes, None)
+
+
+BASE = dict(B=1, Hq=4, Hkv=2, N=1024, d=64, block=64, k_free=4, local_window=1, n_sink=1)
+
+
+@pytest.mark.parametrize("change,status", [
+    (dict(Hq=3), B.DSA_ERR_INVALID_ARG),          # Hq % Hkv != 0
+    (dict(Hkv=0), B.DSA_ERR_INVALID_ARG),
+    (dict(B=-1), B.DSA_ERR_INVALID_ARG),
+    (dict(k_free=-1), B.DSA_ERR_INVALID_ARG),
+    (dict(local_window=-1), B.DSA_ERR_INVALID_ARG),
+    (dict(n_sink=-2), B.DSA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), B.DSA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), B.DSA_ERR_INVALID_ARG),
+    (dict(attn_kernel=7), B.DSA_ERR_INVALID_ARG),
+    (dict(d=96), B.DSA_ERR_UNSUPPORTED),
+    (dict(block=48), B.DSA_ERR_UNSUPPORTED),
+    (dict(N=1000), B.DSA_ERR_UNSUPPORTED),         # N % block != 0
+    (dict(N=32 * 1025, block=32), B.DSA_ERR_UNSUPPORTED),  # nb > 1024
+])
+def test_invalid_params_rejected_before_any_launch(change, status):
+    p = B.Params(**(BASE | change))
+    assert status_of_forward(p) == status
+    n = ctypes.c_size_t(0)
+    assert B.raw("dsa_workspace_size")(p.ref, ctypes.byref(n)) == status
+    assert B.dsa_kmax(p) == 0
+
+
+def test_negative_per_head_budget_rejected():
+    p = B.Params(**BASE, k_per_head=[1, 2, -1, 3])
+    assert status_of_forward(p) == B.DSA_ERR_INVALID_ARG
+    p = B.Params(**(BASE | dict(Hq=512, Hkv=2)), k_per_head=[1] * 512)
+    assert status_of_forward(p) == B.DSA_ERR_UNSUPPORTED
+
+
+def test_null_and_misaligned_pointers_rejected():
+    p = B.Params(**BASE)
+    assert status_of_forward(p, q=None) == B.DSA_ERR_INVALID_ARG
+    assert status_of_forward(p, v=FAKE + 2) == B.DSA_ERR_INVALID_ARG
+    assert status_of_forward(p, out=None) == B.DSA_ERR_INVALID_ARG
+    assert status_of_forward(p, idx=FAKE, cnt=None) == B.DSA_ERR_INVALID_ARG
+    f = B.raw("dsa_sparse_attn_fwd")
+    assert f(p.ref, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, FAKE, 1 << 40, None) == B.DSA_ERR_INVALID_ARG
+    f = B.raw("dsa_block_scores")
+    assert f(p.ref, FAKE, FAKE, None, FAKE, 1 << 40, None) == B.DSA_ERR_INVALID_ARG
+    f = B.raw("dsa_topk_select")
+    assert f(p.ref, FAKE, None, FAKE, None) == B.DSA_ERR_INVALID_ARG
+    assert B.raw("dsa_kmax")(None) == 0
+    assert B.raw("dsa_forward")(None, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, 1, None) \
+        == B.DSA_ERR_INVALID_ARG
+
+
+def test_workspace_checks():
+    p = B.Params(**BASE)
+    need = B.dsa_workspace_size(p)
+    assert status_of_forward(p, ws=None) == B.DSA_ERR_WORKSPACE
+    assert status_of_forward(p, ws_bytes=need - 1) == B.DSA_ERR_WORKSPACE
+    assert status_of_forward(p, ws=FAKE + 8) == B.DSA_ERR_WORKSPACE
+    assert B.raw("dsa_workspace_init")(None, 256, None) == B.DSA_ERR_WORKSPACE
+    assert B.raw("dsa_workspace_init")(FAKE, 100, None) == B.DSA_ERR_WORKSPACE
+    assert B.raw("dsa_check_status")(None, None) == B.DSA_ERR_WORKSPACE
+
+
+def test_empty_problems_return_ok_without_touching_pointers():
+    for change in (dict(B=0), dict(N=0)):
+        p = B.Params(**(BASE | change))
+        assert status_of_forward(p, q=None, k=None, v=None, out=None, ws=None) == B.DSA_OK
+        assert B.dsa_workspace_size(p) == 256
+        assert B.dsa_kmax(p) == 0

@@ -1,0 +1,212 @@
+"""GPU parity: every step of the CUDA path against the fp64 oracle, through the C ABI.
+
+Small cases span several tiles and ragged tails (nb not a multiple of the
+32-lane selection warp, odd block counts, per-head budgets, empty rows); the
+full-size workloads are checked in the launch configuration the benchmark
+uses, on the whole selection and on sampled query blocks of the attention.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dynamic_block_sparse_02_b200 import WORKLOADS, Workload, binding as B
+from dynamic_block_sparse_02_b200 import workloads as W
+from dynamic_block_sparse_02_b200.attention import BlockSparseAttention
+
+from parity import (assert_attention_close, assert_lse_close, compare_selection, dev_bf16,
+                    dev_i32)
+
+pytestmark = pytest.mark.gpu
+
+KERNELS = [B.DSA_ATTN_AUTO, B.DSA_ATTN_MMA_SYNC]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def need_cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    torch.cuda.set_device(0)
+
+
+# name: (B, Hq, Hkv, N, d, block, k_free, local_window, n_sink, k_per_head)
+SMALL = {
+    "tiny-mha": (1, 2, 2, 512, 64, 64, 3, 1, 0, None),
+    "gqa-d128-bs64-ragged": (2, 8, 2, 64 * 37, 128, 64, 5, 2, 1, None),
+    "gqa-d128-bs128": (1, 4, 1, 128 * 21, 128, 128, 4, 1, 0, None),
+    "mha-d64-bs32-perhead": (2, 4, 4, 32 * 45, 64, 32, 0, 1, 0, [1, 2, 4, 8]),
+    "d64-bs128": (1, 2, 1, 128 * 9, 64, 128, 2, 1, 1, None),
+    "d128-bs32": (1, 4, 2, 32 * 70, 128, 32, 6, 1, 2, None),
+    "d64-bs64-g8": (1, 8, 1, 64 * 33, 64, 64, 3, 3, 0, None),
+    "dense": (1, 2, 1, 64 * 12, 128, 64, 1000, 1, 0, None),
+    "empty-rows": (1, 2, 2, 64 * 5, 64, 64, 0, 0, 0, None),
+    "window-only": (1, 2, 1, 64 * 10, 128, 64, 0, 3, 0, None),
+    "sinks-no-window": (1, 2, 2, 32 * 40, 64, 32, 3, 0, 4, None),
+    "nb-1024": (1, 1, 1, 32 * 1024, 64, 32, 7, 1, 1, None),
+}
+
+
+def spec_workload(name):
+    Bn, Hq, Hkv, N, d, bs, k, w, ns, kph = SMALL[name]
+    return Workload(name, Bn, Hq, Hkv, N, d, bs, k_free=k, local_window=w, n_sink=ns), kph
+
+
+def oracle_reference(w, x, kph):
+    qp = oracle.pool_blocks(x["q"], w.block)
+    kp = oracle.pool_blocks(x["k"], w.block)
+    s = oracle.block_scores(qp, kp)
+    k = kph if kph is not None else w.k_free
+    idx, cnt = oracle.select_blocks(s, k, w.local_window, w.n_sink)
+    return s, idx, cnt
+
+
+def per_head(w, kph):
+    return kph if kph is not None else [w.k_free] * w.Hq
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_case_all_steps(name):
+    w, kph = spec_workload(name)
+    x = W.make_inputs(w, seed=7)
+    s64, idx_ref, cnt_ref = oracle_reference(w, x, kph)
+    o_ref, lse_ref = oracle.sparse_attention(x["q"], x["k"], x["v"], idx_ref, cnt_ref, w.block)
+
+    q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+    att = BlockSparseAttention.from_workload(w, k_per_head=kph)
+    # steps 1-2: block scores
+    sc = att.block_scores(q, k)
+    sc_h = sc.cpu().numpy().astype(np.float64)
+    tri = np.tril(np.ones((w.nb, w.nb), dtype=bool))
+    assert np.all(np.isneginf(sc_h[..., ~tri]))
+    np.testing.assert_allclose(sc_h[..., tri], s64[..., tri], rtol=1e-5, atol=1e-6)
+    # step 3 on the GPU's scores, against the oracle's selection
+    idx_s, cnt_s = att.topk_select(sc)
+    idx_s, cnt_s = idx_s.cpu().numpy(), cnt_s.cpu().numpy()
+    n, ties, bad = compare_selection(idx_s, cnt_s, idx_ref, cnt_ref, s64, per_head(w, kph),
+                                     w.local_window, w.n_sink)
+    assert not bad, bad[:5]
+    # fused path: identical selection to the split path, bit for bit
+    idx_f, cnt_f = att.empty_selection()
+    out_f, lse_f = att.empty_out(), att.empty_lse()
+    att.forward(q, k, v, out_f, lse_f, idx_f, cnt_f)
+    np.testing.assert_array_equal(idx_f.cpu().numpy(), idx_s)
+    np.testing.assert_array_equal(cnt_f.cpu().numpy(), cnt_s)
+    # step 4 on the oracle's selection, with each attention kernel
+    for kern in KERNELS:
+        a2 = BlockSparseAttention.from_workload(w, k_per_head=kph, attn_kernel=kern)
+        out, lse = a2.empty_out(), a2.empty_lse()
+        a2.sparse_attn(q, k, v, dev_i32(idx_ref), dev_i32(cnt_ref), out, lse)
+        assert a2.check_status() == B.DSA_OK
+        assert_attention_close(out.double().cpu().numpy(), o_ref, f"{name} kernel {kern}")
+        assert_lse_close(lse.cpu().numpy().astype(np.float64), lse_ref, f"{name} kernel {kern}")
+    # the fused path's output, on rows whose selection equals the oracle's
+    same = (idx_s == idx_ref).all(axis=-1)
+    rows = np.repeat(same, w.block, axis=-1)
+    o_f = out_f.double().cpu().numpy()
+    assert_attention_close(o_f[rows], o_ref[rows], f"{name} fused")
+    assert att.check_status() == B.DSA_OK
+
+
+@pytest.mark.parametrize("kern", KERNELS)
+def test_ones_value_gives_ones(kern):
+    w = Workload("ones", 1, 4, 2, 64 * 20, 128, 64, k_free=3, local_window=2, n_sink=1)
+    x = W.make_inputs(w, seed=3, tensors=("q", "k"))
+    x["q"] = W.f32_to_bf16_bits(W.bf16_bits_to_f32(x["q"]) * 4)  # sharper softmax
+    q, k = dev_bf16(x["q"]), dev_bf16(x["k"])
+    v = torch.ones((w.B, w.Hkv, w.N, w.d), dtype=torch.bfloat16, device="cuda")
+    att = BlockSparseAttention.from_workload(w, attn_kernel=kern)
+    out = att.forward(q, k, v)
+    assert torch.all(out == 1.0)
+    assert att.check_status() == B.DSA_OK
+
+
+def test_out_of_range_index_is_skipped_and_flagged():
+    w = Workload("bad-idx", 1, 2, 2, 64 * 8, 64, 64, k_free=2, local_window=1, n_sink=0)
+    x = W.make_inputs(w, seed=5)
+    s64, idx_ref, cnt_ref = oracle_reference(w, x, None)
+    bad_idx = idx_ref.copy()
+    bad_idx[0, 1, 5, 0] = 7   # a future block (j > i)
+    bad_idx[0, 0, 3, 1] = -4  # negative
+    att = BlockSparseAttention.from_workload(w)
+    q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+    for kern in KERNELS:
+        a2 = BlockSparseAttention.from_workload(w, attn_kernel=kern)
+        out = a2.sparse_attn(q, k, v, dev_i32(bad_idx), dev_i32(cnt_ref))
+        assert a2.check_status() == B.DSA_ERR_DEVICE_BOUNDS
+        assert a2.check_status() == B.DSA_OK  # the flag clears once read
+        # the row without the bad entry matches the oracle on the cleaned list
+        clean = idx_ref.copy()
+        o_ref, _ = oracle.sparse_attention(x["q"], x["k"], x["v"], clean, cnt_ref, w.block)
+        o = out.double().cpu().numpy()
+        assert_attention_close(o[0, 1, :5 * 64], o_ref[0, 1, :5 * 64], "untouched rows")
+    del att
+
+
+def test_cuda_graph_capture_replays_forward():
+    w = WORKLOADS["tiny"]
+    x = W.make_inputs(w)
+    q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+    att = BlockSparseAttention.from_workload(w)
+    ref = att.forward(q, k, v).clone()
+    out = att.empty_out()
+    s = torch.cuda.Stream()
+    att.stream = s
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        att.forward(q, k, v, out)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+
+
+# ---------------------------------------------------------------------------
+# Full-size workloads, in the benchmark's launch configuration (dsa_forward).
+# ---------------------------------------------------------------------------
+
+def sample_items(w, n, seed):
+    g = np.random.default_rng(seed)
+    items = {(int(g.integers(w.B)), int(g.integers(w.Hq)), int(g.integers(w.nb))) for _ in range(n)}
+    for h in range(0, w.Hq, max(1, w.Hq // 4)):
+        items.add((w.B - 1, h, w.nb - 1))
+        items.add((0, h, 0))
+    return sorted(items)
+
+
+@pytest.mark.parametrize("name", ["tiny", "8k-gqa", "32k-gqa", "128k-structured", "batched-32"])
+def test_full_workload(name):
+    w = WORKLOADS[name]
+    kph = W.per_head_k(w)
+    kph_l = None if kph is None else [int(t) for t in kph]
+    x = W.make_inputs(w)
+    s64, idx_ref, cnt_ref = oracle_reference(w, x, kph_l)
+
+    q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+    att = BlockSparseAttention.from_workload(w, k_per_head=kph_l)
+    idx_g, cnt_g = att.empty_selection()
+    out, lse = att.empty_out(), att.empty_lse()
+    att.forward(q, k, v, out, lse, idx_g, cnt_g)
+    assert att.check_status() == B.DSA_OK
+    idx_h, cnt_h = idx_g.cpu().numpy(), cnt_g.cpu().numpy()
+    n, ties, bad = compare_selection(idx_h, cnt_h, idx_ref, cnt_ref, s64, per_head(w, kph_l),
+                                     w.local_window, w.n_sink)
+    print(f"{name}: {n} rows, {ties} near-tie rows, {len(bad)} mismatches")
+    assert not bad, bad[:5]
+
+    items = sample_items(w, 24 if w.N >= 32768 else 64, seed=11)
+    ref = oracle.sparse_attention(x["q"], x["k"], x["v"], idx_ref, cnt_ref, w.block, items=items)
+    out2, lse2 = att.empty_out(), att.empty_lse()
+    att.sparse_attn(q, k, v, dev_i32(idx_ref), dev_i32(cnt_ref), out2, lse2)
+    assert att.check_status() == B.DSA_OK
+    bs = w.block
+    o_g = np.concatenate([out2[b, h, i * bs:(i + 1) * bs].double().cpu().numpy() for (b, h, i) in items])
+    o_r = np.concatenate([ref[it][0] for it in items])
+    assert_attention_close(o_g, o_r, name)
+    l_g = np.concatenate([lse2[b, h, i * bs:(i + 1) * bs].double().cpu().numpy() for (b, h, i) in items])
+    l_r = np.concatenate([ref[it][1] for it in items])
+    assert_lse_close(l_g, l_r, name)
+    # dsa_forward's own output on sampled blocks whose selection equals the oracle's
+    keep = [it for it in items if np.array_equal(idx_h[it], idx_ref[it])]
+    o_f = np.concatenate([out[b, h, i * bs:(i + 1) * bs].double().cpu().numpy() for (b, h, i) in keep])
+    o_r2 = np.concatenate([ref[it][0] for it in keep])
+    assert_attention_close(o_f, o_r2, name + " fused")
