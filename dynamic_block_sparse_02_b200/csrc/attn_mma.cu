@@ -58,6 +58,10 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ float bf16_round(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -117,11 +121,16 @@ attn_mma_kernel(AttnArgs a) {
   __shared__ int sCount;
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int BH = a.B * a.Hq;
-  const int bh = blockIdx.x % BH;
-  const int i = a.nb - 1 - blockIdx.x / BH;  // longest rows first
-  const int b = bh / a.Hq, h = bh % a.Hq;
-  const int kvh = h / a.group;
+  // KV-head-major order (CTAs resident together share one KV head's K/V in
+  // L2); inside a KV head the longest rows (last query blocks) come first.
+  const int per_kv = a.group * a.nb;
+  const int bk = blockIdx.x / per_kv;
+  const int rem = blockIdx.x - bk * per_kv;
+  const int b = bk / a.Hkv;
+  const int kvh = bk - b * a.Hkv;
+  const int i = a.nb - 1 - rem / a.group;
+  const int h = kvh * a.group + rem % a.group;
+  const int bh = b * a.Hq + h;
   const size_t row_id = (size_t)bh * a.nb + i;
 
   // Kept list -> shared memory, dropping out-of-range entries (flagged).
@@ -233,13 +242,14 @@ attn_mma_kernel(AttnArgs a) {
     const float al0 = ex2(m0 - mu0), al1 = ex2(m1 - mu1);
     m0 = mn0;
     m1 = mn1;
+    // P in bf16 (the MMA's input); row sums are taken over the same bf16 values
     float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
     for (int t = 0; t < NT_S; ++t) {
-      s[t][0] = ex2(s[t][0] - mu0);
-      s[t][1] = ex2(s[t][1] - mu0);
-      s[t][2] = ex2(s[t][2] - mu1);
-      s[t][3] = ex2(s[t][3] - mu1);
+      s[t][0] = bf16_round(ex2(s[t][0] - mu0));
+      s[t][1] = bf16_round(ex2(s[t][1] - mu0));
+      s[t][2] = bf16_round(ex2(s[t][2] - mu1));
+      s[t][3] = bf16_round(ex2(s[t][3] - mu1));
       ps0 += s[t][0] + s[t][1];
       ps1 += s[t][2] + s[t][3];
     }

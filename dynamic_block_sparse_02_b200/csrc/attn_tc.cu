@@ -1,15 +1,779 @@
-// Block-sparse attention forward on tcgen05 tensor cores (placeholder until
-// the kernel lands: reports the shape as unsupported).
+// Block-sparse causal attention forward (step 4) on the 5th-generation tensor
+// cores (tcgen05 + TMEM + TMA), for 64x64 blocks and head dim 128.
+//
+// What it computes is the same as the warp-MMA kernel: for every query block
+// i of (b, query head h), softmax(Q K^T * scale) V over the kept key blocks
+// only, causal inside the diagonal block, with K/V of KV head h / (Hq/Hkv)
+// ("稀疏注意力 vs Flash Attention v2", section 1; FlashAttention-style online
+// softmax; "DeepSeek NSA", section 2.2, bf16 matmul with fp32 accumulation).
+//
+// Shape of the computation on sm_100a. A query block has only 64 rows, and
+// every (head, query block) keeps its own list of key blocks, so stacking
+// two query blocks into one 128-row MMA would multiply masked work. Instead
+// the kernel computes transposed products whose 128-row side is the keys of
+// two kept blocks:
+//     S^T (128 keys x 64 queries) = K_pair (128 x d) . Q^T        (M=128, N=64)
+//     O^T (d=128 x 64 queries)   += V_pair^T (128 x 128 keys) . P^T (M=128, N=64)
+// so every tcgen05.mma runs at M=128 without any wasted rows. In TMEM a
+// thread of the softmax warpgroup owns one key (lane) of S^T and one head-dim
+// row of O^T. The softmax maximum is per query (a TMEM column), i.e. across
+// threads; it is kept as a running value per query that is only raised when
+// some logit exceeds it by more than 2^8 (checked by a CTA-wide vote), which
+// keeps P in [0, 2^8] and makes the cross-thread reduction and the rescale of
+// O rare events. The row sums are kept per thread and reduced once per query
+// block.
+//
+// Warp roles (256 threads, one persistent CTA per SM):
+//   warp 0      TMA producer: work items, kept lists, Q / K / V tile loads
+//   warp 1      TMEM allocator and single-thread MMA issuer
+//   warps 4-7   softmax and epilogue (TMEM lanes 0-127)
+// Work items are taken from a global counter in KV-head-major order (so the
+// CTAs running at one time gather K/V of one KV head, which stays in L2),
+// longest rows first inside a KV head.
+//
+// Every wait on an mbarrier is bounded (about 2 s); on expiry the kernel sets
+// DSA_ERR_DEVICE_TIMEOUT in the workspace header, stops issuing work, drains
+// and returns.
+#include <cuda.h>
+
 #include "dsa_internal.cuh"
 
 namespace dsa {
+namespace {
 
-bool attn_tc_supported(const Shape&) { return false; }
+constexpr int kBS = 64;        // query / key block
+constexpr int kD = 128;        // head dim
+constexpr int kChunk = 128;    // keys per S^T tile (two blocks)
+constexpr int kThreads = 256;
+constexpr float kTau = 8.0f;   // rescale threshold (log2 units)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
-cudaError_t launch_attn_tc(const Shape&, const __nv_bfloat16*, const __nv_bfloat16*,
-                           const __nv_bfloat16*, const int32_t*, const int32_t*, __nv_bfloat16*,
-                           float*, WsHeader*, cudaStream_t) {
-  return cudaErrorNotSupported;
+// Shared memory map (bytes from a 1024-byte aligned base).
+constexpr int kQBytes = kBS * kD * 2;         // 16 KB: [2 d-halves][64 rows][128 B]
+constexpr int kKVBytes = kChunk * kD * 2;     // 32 KB: [2 d-halves][128 rows][128 B]
+constexpr int kPBytes = kChunk * kBS * 2;     // 16 KB: [128 keys][64 queries] bf16
+constexpr int kOffQ = 0;                      // 2 buffers
+constexpr int kOffK = kOffQ + 2 * kQBytes;    // 2 stages
+constexpr int kOffV = kOffK + 2 * kKVBytes;   // 2 stages
+constexpr int kOffP = kOffV + 2 * kKVBytes;   // 2 buffers
+constexpr int kOffList = kOffP + 2 * kPBytes; // kMaxBlocks ints
+constexpr int kOffRed = kOffList + kMaxBlocks * 4;  // 4 x 64 floats
+constexpr int kOffM = kOffRed + 4 * 64 * 4;         // 64 floats (running max)
+constexpr int kOffL = kOffM + 64 * 4;               // 64 floats (row sums)
+constexpr int kOffA = kOffL + 64 * 4;               // 64 floats (rescale factors)
+constexpr int kOffBar = kOffA + 64 * 4;             // mbarriers
+constexpr int kNumBars = 22;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;    // tmem base, abort flag, item slots
+constexpr int kSmemBytes = kOffMisc + 64 + 1024;    // + alignment slack
+
+// barrier indices
+enum {
+  B_ITEM_FULL = 0, B_ITEM_EMPTY = 2, B_Q_FULL = 4, B_Q_EMPTY = 6, B_K_FULL = 8, B_K_EMPTY = 10,
+  B_V_FULL = 12, B_V_EMPTY = 14, B_S_FULL = 16, B_P_FULL = 18, B_P_EMPTY = 20
+};
+
+// TMEM columns: S^T buffers at 0 and 64, O^T at 128.
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS = 0, kColO = 128;
+
+struct ItemSlot {
+  int b, h, i, n, diag_last;
+};
+
+struct TcArgs {
+  const int32_t* idx;
+  const int32_t* cnt;
+  __nv_bfloat16* out;
+  float* lse;
+  WsHeader* hdr;
+  int B, Hq, Hkv, N, nb, W, group;
+  int n_items;
+  float scale_log2;
+};
+
+// ----------------------------------------------------------------------------
+// PTX helpers
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait. Returns false (and raises the CTA abort flag and the device
+// error) when the phase does not complete within the limit, or at once when
+// the CTA is already aborting.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       WsHeader* hdr, int where) {
+  if (mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = now_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort_flag) return false;
+      if (now_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        raise_error(hdr, DSA_ERR_DEVICE_TIMEOUT, kKernAttnTc, where, (int)blockIdx.x);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 64 consecutive fp32 columns of this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]),
+        "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]),
+        "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+        "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]),
+        "=r"(r[63])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,"
+      "%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
+      "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+      "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]),
+      "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]),
+      "r"(r[30]), "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]),
+      "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]),
+      "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]), "r"(r[50]),
+      "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]), "r"(r[57]),
+      "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void add_bf16_pair(float& lo, float& hi, uint32_t w) {
+  lo += __uint_as_float(w << 16);
+  hi += __uint_as_float(w & 0xffff0000u);
+}
+
+// Named barrier over the 128 softmax threads (id 1), optionally OR-reducing a predicate.
+__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ bool softmax_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+
+// Shared-memory matrix descriptor (sm_100 format, 128-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor: bf16 x bf16 -> fp32, M=128, N=64.
+constexpr uint32_t idesc_mn(uint32_t a_mn_major, uint32_t b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn_major << 15) | (b_mn_major << 16) |
+         ((uint32_t)(kBS >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+constexpr uint32_t kIdescS = idesc_mn(0, 0);   // A = K (K-major), B = Q (K-major)
+constexpr uint32_t kIdescPV = idesc_mn(1, 1);  // A = V^T (MN-major), B = P^T (MN-major)
+
+// Column-wise reductions over the 32 lanes of a warp for 64 columns held one
+// per register: after the call, v[0] and v[1] hold the reduced values of
+// columns col0 and col0+1, col0 = 2 * (bit-reversed pattern of the lane).
+template <bool kMax>
+__device__ __forceinline__ int warp_col_reduce(float (&v)[64], int lane) {
+#define DSA_RED(OFF, HALF)                                                     \
+  {                                                                            \
+    const bool up = (lane & OFF) != 0;                                         \
+    _Pragma("unroll") for (int j = 0; j < HALF; ++j) {                         \
+      const float send = up ? v[j] : v[j + HALF];                              \
+      const float keep = up ? v[j + HALF] : v[j];                              \
+      const float got = __shfl_xor_sync(0xffffffffu, send, OFF);               \
+      v[j] = kMax ? fmaxf(keep, got) : (keep + got);                           \
+    }                                                                          \
+  }
+  DSA_RED(16, 32)
+  DSA_RED(8, 16)
+  DSA_RED(4, 8)
+  DSA_RED(2, 4)
+  DSA_RED(1, 2)
+#undef DSA_RED
+  return ((lane >> 4) & 1) * 32 + ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 +
+         ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
+}
+
+__device__ __forceinline__ void decode_item(const TcArgs& a, int item, int& b, int& h, int& i) {
+  // KV-head-major; inside a KV head, query blocks from the last (longest) down;
+  // the group's query heads interleaved.
+  const int per_kv = a.group * a.nb;
+  const int bk = item / per_kv;
+  const int rem = item - bk * per_kv;
+  b = bk / a.Hkv;
+  const int kvh = bk - b * a.Hkv;
+  i = a.nb - 1 - rem / a.group;
+  h = kvh * a.group + rem % a.group;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  int* sList = reinterpret_cast<int*>(smem + kOffList);
+  float* sRed = reinterpret_cast<float*>(smem + kOffRed);
+  float* sM = reinterpret_cast<float*>(smem + kOffM);
+  float* sL = reinterpret_cast<float*>(smem + kOffL);
+  float* sA = reinterpret_cast<float*>(smem + kOffA);
+  const uint32_t bars = sbase + kOffBar;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  ItemSlot* sItem = reinterpret_cast<ItemSlot*>(smem + kOffMisc + 16);  // 2 slots
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  auto bar = [&](int idx) { return bars + 8u * idx; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(B_ITEM_FULL + s), 1);
+      mbar_init(bar(B_ITEM_EMPTY + s), 2);
+      mbar_init(bar(B_Q_FULL + s), 1);
+      mbar_init(bar(B_Q_EMPTY + s), 1);
+      mbar_init(bar(B_K_FULL + s), 1);
+      mbar_init(bar(B_K_EMPTY + s), 1);
+      mbar_init(bar(B_V_FULL + s), 1);
+      mbar_init(bar(B_V_EMPTY + s), 1);
+      mbar_init(bar(B_S_FULL + s), 1);
+      mbar_init(bar(B_P_FULL + s), 128);
+      mbar_init(bar(B_P_EMPTY + s), 1);
+    }
+    *sAbort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(sTmem)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sTmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    uint32_t gq = 0, gk = 0, gv = 0;
+    // per ring: bit 2u set = stage u has an issued load, bit u = that load's phase parity
+    uint32_t lastQ = 0, lastK = 0, lastV = 0;
+    for (int t = 0;; ++t) {
+      const int s = t & 1;
+      bool ok = true;
+      if (lane == 0 && t >= 2) ok = mbar_wait(bar(B_ITEM_EMPTY + s), ((t >> 1) - 1) & 1, sAbort, a.hdr, 1);
+      int item = 0;
+      if (lane == 0) item = (*sAbort) ? a.n_items : (int)atomicAdd(&a.hdr->work[0], 1u);
+      item = __shfl_sync(0xffffffffu, item, 0);
+      if (item >= a.n_items) {
+        if (lane == 0) {
+          sItem[s].n = -1;
+          mbar_arrive(bar(B_ITEM_FULL + s));
+        }
+        break;
+      }
+      int b, h, i;
+      decode_item(a, item, b, h, i);
+      const size_t row_id = ((size_t)b * a.Hq + h) * a.nb + i;
+      int n_raw = a.cnt[row_id];
+      if (n_raw < 0 || n_raw > a.W) {
+        if (lane == 0) raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnTc, (int)row_id, n_raw);
+        n_raw = n_raw < 0 ? 0 : a.W;
+      }
+      const int32_t* lst = a.idx + row_id * a.W;
+      int n = 0;
+      for (int base = 0; base < n_raw; base += 32) {
+        const int t2 = base + lane;
+        int j = t2 < n_raw ? lst[t2] : -1;
+        const bool in = t2 < n_raw;
+        const bool valid = in && j >= 0 && j <= i;
+        if (in && !valid) raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnTc, (int)row_id, j);
+        const uint32_t m = __ballot_sync(0xffffffffu, valid);
+        if (valid) sList[n + __popc(m & ((1u << lane) - 1u))] = j;
+        n += __popc(m);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        sItem[s].b = b;
+        sItem[s].h = h;
+        sItem[s].i = i;
+        sItem[s].n = n;
+        sItem[s].diag_last = (n > 0 && sList[n - 1] == i) ? 1 : 0;
+        mbar_arrive(bar(B_ITEM_FULL + s));
+        if (n > 0 && ok) {
+          const uint32_t qb = gq & 1;
+          if (gq >= 2) ok = mbar_wait(bar(B_Q_EMPTY + qb), ((gq >> 1) - 1) & 1, sAbort, a.hdr, 2);
+          const int qrow = (int)(((size_t)b * a.Hq + h) * a.N + (size_t)i * kBS);
+          if (ok) {
+            mbar_expect_tx(bar(B_Q_FULL + qb), kQBytes);
+            const uint32_t dq = sbase + kOffQ + qb * kQBytes;
+            tma_load_2d(dq, &tmQ, 0, qrow, bar(B_Q_FULL + qb));
+            tma_load_2d(dq + kQBytes / 2, &tmQ, 64, qrow, bar(B_Q_FULL + qb));
+            lastQ = (lastQ & ~(5u << qb)) | (4u << qb) | (((gq >> 1) & 1u) << qb);
+          }
+          ++gq;
+          const int kvrow0 = (int)(((size_t)b * a.Hkv + h / a.group) * a.N);
+          const int C = (n + 1) >> 1;
+          for (int c = 0; c < C && ok; ++c) {
+            const int nblk = min(2, n - 2 * c);
+            const uint32_t ks = gk & 1;
+            if (gk >= 2) ok = mbar_wait(bar(B_K_EMPTY + ks), ((gk >> 1) - 1) & 1, sAbort, a.hdr, 3);
+            if (!ok) break;
+            mbar_expect_tx(bar(B_K_FULL + ks), nblk * (kKVBytes / 2));
+            const uint32_t dk = sbase + kOffK + ks * kKVBytes;
+            for (int bb = 0; bb < nblk; ++bb) {
+              const int row = kvrow0 + sList[2 * c + bb] * kBS;
+              tma_load_2d(dk + bb * (kKVBytes / 4), &tmK, 0, row, bar(B_K_FULL + ks));
+              tma_load_2d(dk + kKVBytes / 2 + bb * (kKVBytes / 4), &tmK, 64, row, bar(B_K_FULL + ks));
+            }
+            lastK = (lastK & ~(5u << ks)) | (4u << ks) | (((gk >> 1) & 1u) << ks);
+            ++gk;
+            const uint32_t vs = gv & 1;
+            if (gv >= 2) ok = mbar_wait(bar(B_V_EMPTY + vs), ((gv >> 1) - 1) & 1, sAbort, a.hdr, 4);
+            if (!ok) break;
+            mbar_expect_tx(bar(B_V_FULL + vs), nblk * (kKVBytes / 2));
+            const uint32_t dv = sbase + kOffV + vs * kKVBytes;
+            for (int bb = 0; bb < nblk; ++bb) {
+              const int row = kvrow0 + sList[2 * c + bb] * kBS;
+              tma_load_2d(dv + bb * (kKVBytes / 4), &tmV, 0, row, bar(B_V_FULL + vs));
+              tma_load_2d(dv + kKVBytes / 2 + bb * (kKVBytes / 4), &tmV, 64, row, bar(B_V_FULL + vs));
+            }
+            lastV = (lastV & ~(5u << vs)) | (4u << vs) | (((gv >> 1) & 1u) << vs);
+            ++gv;
+          }
+        }
+      }
+      __syncwarp();
+    }
+    // drain: every issued load has landed before the CTA may exit
+    if (lane == 0) {
+      volatile int no_abort = 0;
+      for (int u = 0; u < 2; ++u) {
+        if (lastK & (4u << u)) mbar_wait(bar(B_K_FULL + u), (lastK >> u) & 1u, &no_abort, a.hdr, 5);
+        if (lastV & (4u << u)) mbar_wait(bar(B_V_FULL + u), (lastV >> u) & 1u, &no_abort, a.hdr, 5);
+        if (lastQ & (4u << u)) mbar_wait(bar(B_Q_FULL + u), (lastQ >> u) & 1u, &no_abort, a.hdr, 5);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t gq = 0, gk = 0, gv = 0, gs = 0, gp = 0;
+      bool ok = true;
+      auto issue_pv = [&](int c, int n) {
+        const uint32_t pb = gp & 1, vs = gv & 1;
+        ok = ok && mbar_wait(bar(B_P_FULL + pb), (gp >> 1) & 1, sAbort, a.hdr, 10);
+        ok = ok && mbar_wait(bar(B_V_FULL + vs), (gv >> 1) & 1, sAbort, a.hdr, 11);
+        tc_fence_after();
+        if (ok) {
+          const int ksteps = min(2, n - 2 * c) * (kBS / 16);
+          const uint32_t va = sbase + kOffV + vs * kKVBytes;
+          const uint32_t pa = sbase + kOffP + pb * kPBytes;
+          for (int kk = 0; kk < ksteps; ++kk) {
+            const uint64_t adesc = smem_desc(va + kk * 2048, kKVBytes / 2, 1024);
+            const uint64_t bdesc = smem_desc(pa + kk * 2048, kPBytes, 1024);
+            tc_mma(tmem + kColO, adesc, bdesc, kIdescPV, (c > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(bar(B_P_EMPTY + pb));
+        tc_commit(bar(B_V_EMPTY + vs));
+        ++gp;
+        ++gv;
+      };
+      for (int t = 0;; ++t) {
+        const int s = t & 1;
+        if (!mbar_wait(bar(B_ITEM_FULL + s), (t >> 1) & 1, sAbort, a.hdr, 12)) break;
+        const int n = sItem[s].n;
+        mbar_arrive(bar(B_ITEM_EMPTY + s));
+        if (n < 0) break;
+        if (n == 0) continue;
+        const int C = (n + 1) >> 1;
+        const uint32_t qb = gq & 1;
+        ok = ok && mbar_wait(bar(B_Q_FULL + qb), (gq >> 1) & 1, sAbort, a.hdr, 13);
+        for (int c = 0; c < C; ++c) {
+          const uint32_t ks = gk & 1, sb = gs & 1;
+          ok = ok && mbar_wait(bar(B_K_FULL + ks), (gk >> 1) & 1, sAbort, a.hdr, 14);
+          tc_fence_after();
+          if (ok) {
+            const uint32_t ka = sbase + kOffK + ks * kKVBytes;
+            const uint32_t qa = sbase + kOffQ + qb * kQBytes;
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              const uint64_t adesc = smem_desc(ka + (kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32, 16, 1024);
+              const uint64_t bdesc = smem_desc(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024);
+              tc_mma(tmem + kColS + sb * kBS, adesc, bdesc, kIdescS, kk > 0 ? 1u : 0u);
+            }
+          }
+          tc_commit(bar(B_S_FULL + sb));
+          tc_commit(bar(B_K_EMPTY + ks));
+          if (c == C - 1) tc_commit(bar(B_Q_EMPTY + qb));
+          ++gk;
+          ++gs;
+          if (c >= 1) issue_pv(c - 1, n);
+        }
+        issue_pv(C - 1, n);
+        ++gq;
+      }
+      // wait for the last MMAs before TMEM is released
+      volatile int no_abort = 0;
+      if (gp > 0) mbar_wait(bar(B_P_EMPTY + ((gp - 1) & 1)), ((gp - 1) >> 1) & 1, &no_abort, a.hdr, 15);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int sp = warp - 4;            // TMEM sub-partition: lanes 32*sp ..
+    const int r = sp * 32 + lane;       // key row of S^T / head-dim row of O^T
+    const uint32_t lane_addr = (uint32_t)(sp * 32) << 16;
+    const float c2 = a.scale_log2;
+    float l[64];  // this thread's share of the row sums (running maxima live in sM)
+    uint32_t gs = 0, gp = 0;
+    uint32_t pend = 0, ph_empty = 0;  // bit b: P buffer b awaits its PV / parity of its next phase
+    auto wait_pv = [&](uint32_t pb) {
+      if (pend & (1u << pb)) {
+        mbar_wait(bar(B_P_EMPTY + pb), (ph_empty >> pb) & 1u, sAbort, a.hdr, 20);
+        ph_empty ^= 1u << pb;
+        pend &= ~(1u << pb);
+      }
+    };
+    for (int t = 0;; ++t) {
+      const int s = t & 1;
+      mbar_wait(bar(B_ITEM_FULL + s), (t >> 1) & 1, sAbort, a.hdr, 21);
+      const ItemSlot it = sItem[s];
+      // one decision for the whole warpgroup (also orders the slot reads before the release)
+      const bool stop = softmax_any(it.n < 0 || *sAbort != 0);
+      if (threadIdx.x == 128) mbar_arrive(bar(B_ITEM_EMPTY + s));
+      if (stop) break;
+      const int C = (it.n + 1) >> 1;
+#pragma unroll
+      for (int q = 0; q < 64; ++q) l[q] = 0.f;
+      for (int c = 0; c < C; ++c) {
+        const uint32_t sb = gs & 1;
+        const uint32_t s_addr = tmem + lane_addr + kColS + sb * kBS;
+        mbar_wait(bar(B_S_FULL + sb), (gs >> 1) & 1, sAbort, a.hdr, 22);
+        ++gs;
+        tc_fence_after();
+        const int nblk = min(2, it.n - 2 * c);
+        const int blk = r / kBS, kl = r % kBS;
+        const bool valid = blk < nblk;
+        const bool diag = (c == C - 1) && it.diag_last && (blk == nblk - 1);
+        float x[64];
+        auto load_logits = [&]() {
+          uint32_t raw[64];
+          tmem_ld64(s_addr, raw);
+#pragma unroll
+          for (int q = 0; q < 64; ++q) {
+            float v = __uint_as_float(raw[q]) * c2;
+            if (!valid || (diag && kl > q)) v = -INFINITY;
+            x[q] = v;
+          }
+        };
+        load_logits();
+        // the first tile sets the maxima; later tiles raise them only past the threshold
+        bool raise = (c == 0);
+        if (!raise) {
+          float dmax = -INFINITY;
+#pragma unroll
+          for (int q4 = 0; q4 < 16; ++q4) {
+            const float4 mv = reinterpret_cast<const float4*>(sM)[q4];
+            dmax = fmaxf(dmax, fmaxf(fmaxf(x[4 * q4] - mv.x, x[4 * q4 + 1] - mv.y),
+                                     fmaxf(x[4 * q4 + 2] - mv.z, x[4 * q4 + 3] - mv.w)));
+          }
+          raise = softmax_any(dmax > kTau);
+        }
+        if (raise) {
+          const int col0 = warp_col_reduce<true>(x, lane);
+          sRed[sp * 64 + col0] = x[0];
+          sRed[sp * 64 + col0 + 1] = x[1];
+          softmax_sync();
+          if (r < 64) {
+            const float mx = fmaxf(fmaxf(sRed[r], sRed[64 + r]), fmaxf(sRed[128 + r], sRed[192 + r]));
+            const float mo = sM[r];
+            const float mn = (c == 0) ? mx : fmaxf(mo, mx);
+            sA[r] = (c == 0) ? 0.f : ex2(mo - mn);
+            sM[r] = mn;
+          }
+          softmax_sync();
+          if (c > 0) {
+            // O^T must hold every earlier tile's contribution before it is rescaled
+            wait_pv(0);
+            wait_pv(1);
+            tc_fence_after();
+            uint32_t o[64];
+            tmem_ld64(tmem + lane_addr + kColO, o);
+#pragma unroll
+            for (int q = 0; q < 64; ++q) {
+              const float alpha = sA[q];
+              l[q] *= alpha;
+              o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+            }
+            tmem_st64(tmem + lane_addr + kColO, o);
+          }
+          load_logits();
+        }
+        // P = 2^(x - m) in bf16, row r of the MN-major P^T tile
+        const uint32_t pb = gp & 1;
+        wait_pv(pb);
+        uint8_t* prow = smem + kOffP + pb * kPBytes + r * 128;
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          float p[8];
+          const float4 m0 = reinterpret_cast<const float4*>(sM)[2 * cc];
+          const float4 m1 = reinterpret_cast<const float4*>(sM)[2 * cc + 1];
+          const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) p[e] = ex2(x[cc * 8 + e] - mm[e]);
+          uint4 w;
+          w.x = pack_bf16(p[0], p[1]);
+          w.y = pack_bf16(p[2], p[3]);
+          w.z = pack_bf16(p[4], p[5]);
+          w.w = pack_bf16(p[6], p[7]);
+          // row sums of the bf16 values the tensor core multiplies
+          add_bf16_pair(l[cc * 8 + 0], l[cc * 8 + 1], w.x);
+          add_bf16_pair(l[cc * 8 + 2], l[cc * 8 + 3], w.y);
+          add_bf16_pair(l[cc * 8 + 4], l[cc * 8 + 5], w.z);
+          add_bf16_pair(l[cc * 8 + 6], l[cc * 8 + 7], w.w);
+          *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = w;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        mbar_arrive(bar(B_P_FULL + pb));
+        pend |= 1u << pb;
+        ++gp;
+      }
+      // ---------------------------------------------------------------- epilogue
+      wait_pv(0);
+      wait_pv(1);
+      tc_fence_after();
+      warp_col_reduce<false>(l, lane);
+      {
+        const int col0 = ((lane >> 4) & 1) * 32 + ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 +
+                         ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
+        sRed[sp * 64 + col0] = l[0];
+        sRed[sp * 64 + col0 + 1] = l[1];
+      }
+      softmax_sync();
+      if (r < 64) sL[r] = (sRed[r] + sRed[64 + r]) + (sRed[128 + r] + sRed[192 + r]);
+      softmax_sync();
+      const size_t row0 = ((size_t)it.b * a.Hq + it.h) * a.N + (size_t)it.i * kBS;
+      uint8_t* stage = smem + kOffP;  // both P buffers are idle here
+      {
+        uint32_t o[64];
+        if (C > 0) {
+          tmem_ld64(tmem + lane_addr + kColO, o);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 64; ++q) o[q] = 0u;
+        }
+        tc_fence_before();
+#pragma unroll
+        for (int q = 0; q < 64; ++q) {
+          const float lq = sL[q];
+          const float v = lq > 0.f ? __uint_as_float(o[q]) / lq : 0.f;
+          reinterpret_cast<__nv_bfloat16*>(stage)[q * kD + r] = __float2bfloat16_rn(v);
+        }
+      }
+      softmax_sync();
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(stage);
+        uint4* dst = reinterpret_cast<uint4*>(a.out + row0 * kD);
+#pragma unroll
+        for (int e = 0; e < (kBS * kD / 8) / 128; ++e) dst[e * 128 + r] = src[e * 128 + r];
+      }
+      if (a.lse != nullptr && r < 64) {
+        const float lq = sL[r];
+        a.lse[row0 + r] = (C > 0 && lq > 0.f) ? (sM[r] * kLn2 + logf(lq)) : -INFINITY;
+      }
+      softmax_sync();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Host side
+// ----------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a [rows][128] bf16 tensor, 64 x 64 boxes, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, unsigned long long rows) {
+  EncodeTiledFn f = encode_fn();
+  if (f == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kBS};
+  cuuint32_t estr[2] = {1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool attn_tc_supported(const Shape& s) {
+  // TMA row coordinates are 32-bit
+  const unsigned long long rows = (unsigned long long)s.B * s.Hq * s.N;
+  return s.bs == kBS && s.d == kD && rows < (1ull << 31) && encode_fn() != nullptr;
+}
+
+cudaError_t launch_attn_tc(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                           const __nv_bfloat16* v, const int32_t* idx, const int32_t* cnt,
+                           __nv_bfloat16* out, float* lse, WsHeader* hdr, cudaStream_t st) {
+  if (!attn_tc_supported(s)) return cudaErrorNotSupported;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, (unsigned long long)s.B * s.Hq * s.N) ||
+      !make_map(&mk, k, (unsigned long long)s.B * s.Hkv * s.N) ||
+      !make_map(&mv, v, (unsigned long long)s.B * s.Hkv * s.N))
+    return cudaErrorInvalidValue;
+  TcArgs a;
+  a.idx = idx;
+  a.cnt = cnt;
+  a.out = out;
+  a.lse = lse;
+  a.hdr = hdr;
+  a.B = s.B;
+  a.Hq = s.Hq;
+  a.Hkv = s.Hkv;
+  a.N = s.N;
+  a.nb = s.nb;
+  a.W = s.W;
+  a.group = s.group;
+  a.n_items = s.B * s.Hq * s.nb;
+  a.scale_log2 = s.scale * kLog2e;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(&hdr->work[0], 0, sizeof(unsigned int), st);
+  if (e != cudaSuccess) return e;
+  const int grid = a.n_items < sms ? a.n_items : sms;
+  attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, a);
+  return cudaGetLastError();
 }
 
 }  // namespace dsa

@@ -201,7 +201,7 @@ dsa_status dsa_topk_select(const dsa_params* p, const float* scores, int32_t* id
   dsa_status st = make_shape(p, &s);
   if (st != DSA_OK) return st;
   if (is_empty(p)) return DSA_OK;
-  if (scores == nullptr || idx == nullptr || cnt == nullptr || !aligned16(scores))
+  if (scores == nullptr || (idx == nullptr && s.W > 0) || cnt == nullptr || !aligned16(scores))
     return DSA_ERR_INVALID_ARG;
   if ((st = check_device()) != DSA_OK) return st;
   return from_cuda(dsa::launch_select(s, budgets(p), scores, idx, cnt, nullptr, (cudaStream_t)stream));
@@ -213,8 +213,8 @@ dsa_status dsa_select_blocks(const dsa_params* p, const dsa_bf16* q, const dsa_b
   dsa_status st = make_shape(p, &s);
   if (st != DSA_OK) return st;
   if (is_empty(p)) return DSA_OK;
-  if (q == nullptr || k == nullptr || idx == nullptr || cnt == nullptr || !aligned16(q) ||
-      !aligned16(k))
+  if (q == nullptr || k == nullptr || (idx == nullptr && s.W > 0) || cnt == nullptr ||
+      !aligned16(q) || !aligned16(k))
     return DSA_ERR_INVALID_ARG;
   if ((st = check_ws(s, ws, ws_bytes)) != DSA_OK) return st;
   if ((st = check_device()) != DSA_OK) return st;
@@ -228,8 +228,9 @@ dsa_status dsa_sparse_attn_fwd(const dsa_params* p, const dsa_bf16* q, const dsa
   dsa_status st = make_shape(p, &s);
   if (st != DSA_OK) return st;
   if (is_empty(p)) return DSA_OK;
-  if (q == nullptr || k == nullptr || v == nullptr || idx == nullptr || cnt == nullptr ||
-      out == nullptr || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+  if (q == nullptr || k == nullptr || v == nullptr || (idx == nullptr && s.W > 0) ||
+      cnt == nullptr || out == nullptr || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      !aligned16(out))
     return DSA_ERR_INVALID_ARG;
   if ((st = check_ws(s, ws, ws_bytes)) != DSA_OK) return st;
   if ((st = check_device()) != DSA_OK) return st;
@@ -247,13 +248,15 @@ dsa_status dsa_forward(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || !aligned16(q) ||
       !aligned16(k) || !aligned16(v) || !aligned16(out))
     return DSA_ERR_INVALID_ARG;
-  if ((idx == nullptr) != (cnt == nullptr)) return DSA_ERR_INVALID_ARG;
+  // idx may be NULL alongside a caller cnt only when rows hold no entries (W == 0)
+  if (cnt == nullptr && idx != nullptr) return DSA_ERR_INVALID_ARG;
+  if (cnt != nullptr && idx == nullptr && s.W > 0) return DSA_ERR_INVALID_ARG;
   if ((st = check_ws(s, ws, ws_bytes)) != DSA_OK) return st;
   if ((st = check_device()) != DSA_OK) return st;
   const Layout L = layout(s);
   char* base = static_cast<char*>(ws);
   auto hdr = reinterpret_cast<dsa::WsHeader*>(base);
-  if (idx == nullptr) {
+  if (cnt == nullptr) {
     idx = reinterpret_cast<int32_t*>(base + L.idx);
     cnt = reinterpret_cast<int32_t*>(base + L.cnt);
   }

@@ -129,16 +129,25 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
 
 // ---------------------------------------------------------------------------
 // Step 3: selection of one row (b, h, i) by one warp.
-// s: the row's scores s[0..i] (shared memory). Writes idx_row[0..W) (kept
-// blocks ascending, then -1) and *cnt_out.
+// s: the row's scores s[0..i] (shared memory); skey: per-warp scratch of at
+// least i+1 words. Writes idx_row[0..W) (kept blocks ascending, then -1) and
+// *cnt_out.
 //
-// The k best candidates are found by a most-significant-bit-first radix
-// select on the ordered keys: after each bit the warp knows how many
-// candidates share the current key prefix; it stops once that many are still
-// needed, or after bit 0, in which case the remaining picks are the lowest
-// block indices among equal keys.
+// Candidates are the causal blocks outside the forced set; lane l owns blocks
+// l, l+32, l+64, ... The k best (larger fp32 score first, lower block index on
+// ties) are found in three steps:
+//  1. a lower bound L on the k-th best key: with r = ceil(k/32), every lane's
+//     r-th largest key is >= the minimum of those over the warp, so at least
+//     32r >= k keys are >= L (L = 0, no bound, when some lane has fewer than
+//     r candidates or r > 4);
+//  2. the candidates with key >= L ("survivors") are compacted into skey;
+//  3. a most-significant-bit-first radix select over the survivors, starting
+//     at the highest bit in which they differ, finds the threshold prefix;
+//     equal keys left at the end are taken in increasing block index.
 // ---------------------------------------------------------------------------
-__device__ void select_row(const float* s, int i, int k, int lw, int ns, int W,
+__device__ __forceinline__ bool is_forced(int j, int win_lo, int ns) { return j >= win_lo || j < ns; }
+
+__device__ void select_row(const float* s, uint32_t* skey, int i, int k, int lw, int ns, int W,
                            int32_t* __restrict__ idx_row, int32_t* __restrict__ cnt_out,
                            WsHeader* hdr, int lane) {
   const int n = i + 1;
@@ -147,62 +156,107 @@ __device__ void select_row(const float* s, int i, int k, int lw, int ns, int W,
   const int ncand = n - nforced;
   const int keff = min(k, ncand);
   const int T = (n + 31) >> 5;
-
-  uint32_t key[kMaxBlocks / 32];
-#pragma unroll
-  for (int t = 0; t < kMaxBlocks / 32; ++t) {
-    const int j = t * 32 + lane;
-    uint32_t kk = 0;
-    if (t < T && j < n && !(j >= win_lo || j < ns)) kk = ordered_key(s[j]);
-    key[t] = kk;
-  }
-
-  uint32_t prefix = 0, pmask = 0;
-  int need = keff, m = ncand;
-  for (int bit = 31; bit >= 0 && need > 0 && m != need; --bit) {
-    const uint32_t bb = 1u << bit;
-    int c = 0;
-#pragma unroll
-    for (int t = 0; t < kMaxBlocks / 32; ++t)
-      if (t < T)
-        c += (key[t] != 0u) & ((key[t] & pmask) == prefix) & ((key[t] & bb) != 0u);
-    c = __reduce_add_sync(kFull, c);
-    if (c >= need) {
-      prefix |= bb;
-      m = c;
-    } else {
-      need -= c;
-      m -= c;
-    }
-    pmask |= bb;
-  }
-
   const uint32_t lt = (1u << lane) - 1u;
-  int base = 0, rank_base = 0;
-#pragma unroll
-  for (int t = 0; t < kMaxBlocks / 32; ++t) {
-    if (t < T) {
-      const int j = t * 32 + lane;
-      const bool forced = j < n && (j >= win_lo || j < ns);
-      const uint32_t kk = key[t];
-      const bool valid = kk != 0u;
-      const bool above = valid && ((kk & pmask) > prefix);
-      const bool match = valid && ((kk & pmask) == prefix);
-      const uint32_t mm = __ballot_sync(kFull, match);
-      const int r = rank_base + __popc(mm & lt);
-      rank_base += __popc(mm);
-      const bool sel = forced || above || (match && r < need);
-      const uint32_t sm = __ballot_sync(kFull, sel);
-      const int pos = base + __popc(sm & lt);
-      if (sel) {
-        if (pos < W) idx_row[pos] = j;
-        else raise_error(hdr, DSA_ERR_DEVICE_BOUNDS, kKernSelect, i, pos);
+
+  uint32_t surv = 0;          // bit t: block lane + 32t is a survivor
+  uint32_t prefix = 0, pmask = 0;
+  int need = keff;
+  if (keff > 0 && keff < ncand) {
+    // 1. lower bound from each lane's r-th largest key
+    const int r = (keff + 31) >> 5;
+    uint32_t L = 0;
+    if (r <= 4) {
+      uint32_t t0 = 0, t1 = 0, t2 = 0, t3 = 0;  // this lane's largest keys, descending
+      for (int t = 0; t < T; ++t) {
+        const int j = t * 32 + lane;
+        if (j < n && !is_forced(j, win_lo, ns)) {
+          uint32_t v = ordered_key(s[j]), u;
+          u = max(t0, v); v = min(t0, v); t0 = u;
+          u = max(t1, v); v = min(t1, v); t1 = u;
+          u = max(t2, v); v = min(t2, v); t2 = u;
+          t3 = max(t3, v);
+        }
       }
-      base += __popc(sm);
+      const uint32_t mine = r == 1 ? t0 : r == 2 ? t1 : r == 3 ? t2 : t3;
+      L = __reduce_min_sync(kFull, mine);
     }
+    // 2. compact the survivors' keys
+    int m = 0;
+    for (int t = 0; t < T; ++t) {
+      const int j = t * 32 + lane;
+      uint32_t key = 0;
+      if (j < n && !is_forced(j, win_lo, ns)) key = ordered_key(s[j]);
+      const bool sv = key != 0u && key >= L;
+      const uint32_t bm = __ballot_sync(kFull, sv);
+      if (sv) skey[m + __popc(bm & lt)] = key;
+      surv |= (uint32_t)sv << t;
+      m += __popc(bm);
+    }
+    __syncwarp();
+    // 3. radix select over the survivors from their highest differing bit
+    const uint32_t k0 = skey[0];
+    uint32_t diff = 0;
+    for (int u = lane; u < m; u += 32) diff |= skey[u] ^ k0;
+    diff = __reduce_or_sync(kFull, diff);
+    if (diff == 0u) {
+      pmask = 0xffffffffu;  // all survivors equal: lowest indices win
+      prefix = k0;
+    } else {
+      const int hb = 31 - __clz(diff);
+      pmask = hb == 31 ? 0u : ~((2u << hb) - 1u);
+      prefix = k0 & pmask;
+      int msurv = m;
+      for (int bit = hb; bit >= 0 && msurv != need; --bit) {
+        const uint32_t bb = 1u << bit;
+        int c = 0;
+        for (int u = lane; u < m; u += 32) {
+          const uint32_t key = skey[u];
+          c += ((key & pmask) == prefix) & ((key & bb) != 0u);
+        }
+        c = __reduce_add_sync(kFull, c);
+        if (c >= need) {
+          prefix |= bb;
+          msurv = c;
+        } else {
+          need -= c;
+          msurv -= c;
+        }
+        pmask |= bb;
+      }
+    }
+  } else if (keff > 0) {
+    // every candidate is kept
+    for (int t = 0; t < T; ++t) {
+      const int j = t * 32 + lane;
+      surv |= (uint32_t)(j < n && !is_forced(j, win_lo, ns)) << t;
+    }
+    need = ncand;  // pmask = prefix = 0: every survivor matches
+  }
+
+  // emit forced blocks and picks in ascending block order
+  int base = 0, rank_base = 0;
+  for (int t = 0; t < T; ++t) {
+    const int j = t * 32 + lane;
+    const bool forced = j < n && is_forced(j, win_lo, ns);
+    const bool sv = (surv >> t) & 1u;
+    const uint32_t key = sv ? ordered_key(s[j]) : 0u;
+    const bool above = sv && ((key & pmask) > prefix);
+    const bool match = sv && ((key & pmask) == prefix);
+    const uint32_t mm = __ballot_sync(kFull, match);
+    const int rk = rank_base + __popc(mm & lt);
+    rank_base += __popc(mm);
+    const bool sel = forced || above || (match && rk < need);
+    const uint32_t sm = __ballot_sync(kFull, sel);
+    const int pos = base + __popc(sm & lt);
+    if (sel) {
+      if (pos < W) idx_row[pos] = j;
+      else raise_error(hdr, DSA_ERR_DEVICE_BOUNDS, kKernSelect, i, pos);
+    }
+    base += __popc(sm);
   }
   for (int p = base + lane; p < W; p += 32) idx_row[p] = -1;
   if (lane == 0) *cnt_out = min(base, W);
+  __syncwarp();
 }
 
 // Rows handled by one CTA of the score kernels: heads [h0, h0+HB) of one KV
@@ -240,6 +294,7 @@ score_kernel(Shape s, KBudget kb, int HB, int RB, const float* __restrict__ qp,
   extern __shared__ float sm_f[];
   float* qs = sm_f;                       // [8][D]
   float* sc = sm_f + kSelWarps * D;       // [8][nb]
+  uint32_t* sk = reinterpret_cast<uint32_t*>(sc + kSelWarps * s.nb);  // [8][nb] (FUSED only)
   const RowTile tile = row_tile(s, HB, RB);
   const int h_end = min(tile.h0 + HB, (tile.kvh + 1) * s.group);
   const int i_end = min(tile.i0 + RB, s.nb);
@@ -275,7 +330,8 @@ score_kernel(Shape s, KBudget kb, int HB, int RB, const float* __restrict__ qp,
   const size_t row = ((size_t)tile.b * s.Hq + h) * s.nb + i;
   if (FUSED) {
     const int k = s.per_head ? kb.k[h] : kb.k[0];
-    select_row(sc + r * s.nb, i, k, s.lw, s.ns, s.W, idx + row * s.W, cnt + row, hdr, lane);
+    select_row(sc + r * s.nb, sk + r * s.nb, i, k, s.lw, s.ns, s.W, idx + row * s.W, cnt + row, hdr,
+               lane);
   } else {
     float* dst = scores + row * s.nb;
     for (int j = lane; j < s.nb; j += 32) dst[j] = (j <= i) ? sc[r * s.nb + j] : -INFINITY;
@@ -293,11 +349,12 @@ select_kernel(Shape s, KBudget kb, const float* __restrict__ scores, int32_t* __
   const int i = (int)(row % s.nb);
   const int h = (int)((row / s.nb) % s.Hq);
   float* sc = sm_f + warp * s.nb;
+  uint32_t* sk = reinterpret_cast<uint32_t*>(sm_f + kSelWarps * s.nb) + warp * s.nb;
   const float* src = scores + (size_t)row * s.nb;
   for (int j = lane; j <= i; j += 32) sc[j] = src[j];
   __syncwarp();
   const int k = s.per_head ? kb.k[h] : kb.k[0];
-  select_row(sc, i, k, s.lw, s.ns, s.W, idx + (size_t)row * s.W, cnt + row, hdr, lane);
+  select_row(sc, sk, i, k, s.lw, s.ns, s.W, idx + (size_t)row * s.W, cnt + row, hdr, lane);
 }
 
 void row_tiling(const Shape& s, int& HB, int& RB) {
@@ -318,7 +375,7 @@ cudaError_t launch_score_impl(const Shape& s, const KBudget& kb, const float* qp
                               cudaStream_t st) {
   int HB, RB;
   row_tiling(s, HB, RB);
-  const size_t smem = (size_t)kSelWarps * (s.d + s.nb) * sizeof(float);
+  const size_t smem = (size_t)kSelWarps * (s.d + (FUSED ? 2 : 1) * s.nb) * sizeof(float);
   const int grid = score_grid(s, HB, RB);
   if (s.d == 64) {
     auto f = score_kernel<64, FUSED>;
@@ -372,7 +429,7 @@ cudaError_t launch_select(const Shape& s, const KBudget& kb, const float* scores
                           int32_t* cnt, WsHeader* hdr, cudaStream_t st) {
   const long long n_rows = (long long)s.B * s.Hq * s.nb;
   const long long grid = (n_rows + kSelWarps - 1) / kSelWarps;
-  const size_t smem = (size_t)kSelWarps * s.nb * sizeof(float);
+  const size_t smem = (size_t)kSelWarps * 2 * s.nb * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

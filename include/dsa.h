@@ -29,7 +29,8 @@
  *     16-byte aligned.
  *   - Block index rows: idx int32 [B, Hq, nb, W] with nb = N / block and
  *     W = dsa_kmax(p); each row lists its kept key blocks in ascending order,
- *     padded with -1; cnt int32 [B, Hq, nb] holds each row's length.
+ *     padded with -1; cnt int32 [B, Hq, nb] holds each row's length. When
+ *     W == 0 (no block can be kept) idx may be NULL.
  *   - The caller owns all memory. The library never allocates device or host
  *     memory; it uses the caller's workspace (dsa_workspace_size bytes).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy

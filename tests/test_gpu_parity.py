@@ -107,6 +107,49 @@ def test_small_case_all_steps(name):
     assert att.check_status() == B.DSA_OK
 
 
+def tc_supported(w):
+    return w.block == 64 and w.d == 128
+
+
+def test_explicit_tcgen05_kernel_or_unsupported():
+    for name in SMALL:
+        w, kph = spec_workload(name)
+        x = W.make_inputs(w, seed=9)
+        s64, idx_ref, cnt_ref = oracle_reference(w, x, kph)
+        att = BlockSparseAttention.from_workload(w, k_per_head=kph, attn_kernel=B.DSA_ATTN_TCGEN05)
+        q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+        if not tc_supported(w):
+            with pytest.raises(B.DsaError) as e:
+                att.sparse_attn(q, k, v, dev_i32(idx_ref), dev_i32(cnt_ref))
+            assert e.value.status == B.DSA_ERR_UNSUPPORTED
+            continue
+        o_ref, lse_ref = oracle.sparse_attention(x["q"], x["k"], x["v"], idx_ref, cnt_ref, w.block)
+        out, lse = att.empty_out(), att.empty_lse()
+        att.sparse_attn(q, k, v, dev_i32(idx_ref), dev_i32(cnt_ref), out, lse)
+        assert att.check_status() == B.DSA_OK
+        assert_attention_close(out.double().cpu().numpy(), o_ref, name + " tcgen05")
+        assert_lse_close(lse.cpu().numpy().astype(np.float64), lse_ref, name + " tcgen05")
+
+
+def test_exact_score_ties_pick_lower_block_index():
+    # Key blocks repeat one of three patterns, so many block scores tie exactly;
+    # the selection must keep the lower block indices among equal scores.
+    w = Workload("ties", 1, 4, 2, 64 * 70, 128, 64, k_free=9, local_window=1, n_sink=1)
+    x = W.make_inputs(w, seed=13)
+    kb = x["k"].reshape(w.B, w.Hkv, w.nb, w.block, w.d)
+    pattern = np.arange(w.nb) % 3
+    x["k"] = np.ascontiguousarray(kb[:, :, pattern]).reshape(w.B, w.Hkv, w.N, w.d)
+    s64, idx_ref, cnt_ref = oracle_reference(w, x, None)
+    att = BlockSparseAttention.from_workload(w)
+    q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+    idx, cnt = att.select_blocks(q, k)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), cnt_ref)
+    np.testing.assert_array_equal(idx.cpu().numpy(), idx_ref)
+    sc = att.block_scores(q, k)
+    idx2, cnt2 = att.topk_select(sc)
+    np.testing.assert_array_equal(idx2.cpu().numpy(), idx_ref)
+
+
 @pytest.mark.parametrize("kern", KERNELS)
 def test_ones_value_gives_ones(kern):
     w = Workload("ones", 1, 4, 2, 64 * 20, 128, 64, k_free=3, local_window=2, n_sink=1)
@@ -120,14 +163,14 @@ def test_ones_value_gives_ones(kern):
     assert att.check_status() == B.DSA_OK
 
 
-def test_out_of_range_index_is_skipped_and_flagged():
-    w = Workload("bad-idx", 1, 2, 2, 64 * 8, 64, 64, k_free=2, local_window=1, n_sink=0)
+@pytest.mark.parametrize("d", [64, 128])
+def test_out_of_range_index_is_skipped_and_flagged(d):
+    w = Workload("bad-idx", 1, 2, 2, 64 * 8, d, 64, k_free=2, local_window=1, n_sink=0)
     x = W.make_inputs(w, seed=5)
     s64, idx_ref, cnt_ref = oracle_reference(w, x, None)
     bad_idx = idx_ref.copy()
     bad_idx[0, 1, 5, 0] = 7   # a future block (j > i)
     bad_idx[0, 0, 3, 1] = -4  # negative
-    att = BlockSparseAttention.from_workload(w)
     q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
     for kern in KERNELS:
         a2 = BlockSparseAttention.from_workload(w, attn_kernel=kern)
@@ -139,7 +182,6 @@ def test_out_of_range_index_is_skipped_and_flagged():
         o_ref, _ = oracle.sparse_attention(x["q"], x["k"], x["v"], clean, cnt_ref, w.block)
         o = out.double().cpu().numpy()
         assert_attention_close(o[0, 1, :5 * 64], o_ref[0, 1, :5 * 64], "untouched rows")
-    del att
 
 
 def test_cuda_graph_capture_replays_forward():
