@@ -14,22 +14,34 @@
 // two kept blocks:
 //     S^T (128 keys x 64 queries) = K_pair (128 x d) . Q^T        (M=128, N=64)
 //     O^T (d=128 x 64 queries)   += V_pair^T (128 x 128 keys) . P^T (M=128, N=64)
-// so every tcgen05.mma runs at M=128 without any wasted rows. In TMEM a
-// thread of the softmax warpgroup owns one key (lane) of S^T and one head-dim
-// row of O^T. The softmax maximum is per query (a TMEM column), i.e. across
-// threads; it is kept as a running value per query that is only raised when
-// some logit exceeds it by more than 2^8 (checked by a CTA-wide vote), which
-// keeps P in [0, 2^8] and makes the cross-thread reduction and the rescale of
-// O rare events. The row sums are kept per thread and reduced once per query
-// block.
+// so every tcgen05.mma runs at M=128 without any wasted rows (at N=64 an MMA
+// reads 6 KB of shared memory per 128x64x16 step, which bounds the tensor
+// pipe at 2/3 of its N>=128 rate). In TMEM a thread of a softmax warpgroup
+// owns one key (lane) of S^T and one head-dim row of O^T. The softmax maximum
+// is per query (a TMEM column), i.e. across threads; it is kept as a running
+// value per query that is only raised when some logit exceeds it by more than
+// 2^8 (decided by a warpgroup vote), which keeps P in [0, 2^8] and makes the
+// cross-thread reduction and the rescale of O rare. Row sums are kept per
+// thread and reduced once per query block.
 //
-// Warp roles (256 threads, one persistent CTA per SM):
-//   warp 0      TMA producer: work items, kept lists, Q / K / V tile loads
-//   warp 1      TMEM allocator and single-thread MMA issuer
-//   warps 4-7   softmax and epilogue (TMEM lanes 0-127)
-// Work items are taken from a global counter in KV-head-major order (so the
-// CTAs running at one time gather K/V of one KV head, which stays in L2),
-// longest rows first inside a KV head.
+// Warp roles (384 threads, one persistent CTA per SM):
+//   warp 0        TMA producer: work items, kept lists, Q and K tiles
+//   warp 1        issues S^T = K Q^T      (one thread)
+//   warp 2        issues O^T += V^T P^T   (one thread)
+//   warp 3        TMA producer of the V tiles
+//   warps 4-7     softmax + epilogue of stream 0
+//   warps 8-11    softmax + epilogue of stream 1
+// A single issuing thread cannot issue N=64 MMAs as fast as the tensor core
+// retires them, nor tensor-TMA loads as fast as L2 fills shared memory, so the
+// two products and the K and V loads each come from their own warp. Two streams of work
+// items (each with its own Q tile, TMEM S buffers, O accumulator and P tile)
+// alternate chunk by chunk, so that one stream's softmax, rescale and
+// epilogue overlap the other stream's MMAs. The producer and both issuers walk
+// the same deterministic interleaving of (stream, chunk) steps, which is also
+// the order of the shared K and V rings.
+// Work items come from a global counter in KV-head-major order (the CTAs
+// running at one time gather K/V of one KV head, which stays in L2), longest
+// rows first inside a KV head.
 //
 // Every wait on an mbarrier is bounded (about 2 s); on expiry the kernel sets
 // DSA_ERR_DEVICE_TIMEOUT in the workspace header, stops issuing work, drains
@@ -44,7 +56,8 @@ namespace {
 constexpr int kBS = 64;        // query / key block
 constexpr int kD = 128;        // head dim
 constexpr int kChunk = 128;    // keys per S^T tile (two blocks)
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
+constexpr int kStreams = 2;
 constexpr float kTau = 8.0f;   // rescale threshold (log2 units)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -54,29 +67,42 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr int kQBytes = kBS * kD * 2;         // 16 KB: [2 d-halves][64 rows][128 B]
 constexpr int kKVBytes = kChunk * kD * 2;     // 32 KB: [2 d-halves][128 rows][128 B]
 constexpr int kPBytes = kChunk * kBS * 2;     // 16 KB: [128 keys][64 queries] bf16
-constexpr int kOffQ = 0;                      // 2 buffers
-constexpr int kOffK = kOffQ + 2 * kQBytes;    // 2 stages
-constexpr int kOffV = kOffK + 2 * kKVBytes;   // 2 stages
-constexpr int kOffP = kOffV + 2 * kKVBytes;   // 2 buffers
-constexpr int kOffList = kOffP + 2 * kPBytes; // kMaxBlocks ints
-constexpr int kOffRed = kOffList + kMaxBlocks * 4;  // 4 x 64 floats
-constexpr int kOffM = kOffRed + 4 * 64 * 4;         // 64 floats (running max)
-constexpr int kOffL = kOffM + 64 * 4;               // 64 floats (row sums)
-constexpr int kOffA = kOffL + 64 * 4;               // 64 floats (rescale factors)
-constexpr int kOffBar = kOffA + 64 * 4;             // mbarriers
-constexpr int kNumBars = 22;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;    // tmem base, abort flag, item slots
-constexpr int kSmemBytes = kOffMisc + 64 + 1024;    // + alignment slack
+constexpr int kOffQ = 0;                                  // one per stream
+constexpr int kOffK = kOffQ + kStreams * kQBytes;         // 2 ring stages
+constexpr int kOffV = kOffK + 2 * kKVBytes;               // 2 ring stages
+constexpr int kOffP = kOffV + 2 * kKVBytes;               // one per stream
+constexpr int kOffList = kOffP + kStreams * kPBytes;      // [stream][slot][kMaxBlocks] int16
+constexpr int kOffRed = kOffList + kStreams * 2 * kMaxBlocks * 2;  // [stream][4][64] f32
+constexpr int kOffM = kOffRed + kStreams * 4 * 64 * 4;    // [stream][64] running max
+constexpr int kOffL = kOffM + kStreams * 64 * 4;          // [stream][64] 1 / row sum
+constexpr int kOffA = kOffL + kStreams * 64 * 4;          // [stream][64] max increments
+constexpr int kOffT = kOffA + kStreams * 64 * 4;          // [stream][64] raise thresholds on S
+constexpr int kOffBar = kOffT + kStreams * 64 * 4;        // mbarriers
+constexpr int kNumBars = 32;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;          // tmem base, abort flag, item slots
+constexpr int kSmemBytes = kOffMisc + 128 + 1024;         // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-// barrier indices
+// barrier indices ([stream] or [stream][slot|buffer] or [stage])
 enum {
-  B_ITEM_FULL = 0, B_ITEM_EMPTY = 2, B_Q_FULL = 4, B_Q_EMPTY = 6, B_K_FULL = 8, B_K_EMPTY = 10,
-  B_V_FULL = 12, B_V_EMPTY = 14, B_S_FULL = 16, B_P_FULL = 18, B_P_EMPTY = 20
+  B_ITEM_FULL = 0,    // [2][2]
+  B_ITEM_EMPTY = 4,   // [2][2]
+  B_Q_FULL = 8,       // [2]
+  B_Q_EMPTY = 10,     // [2]
+  B_K_FULL = 12,      // [2]
+  B_K_EMPTY = 14,     // [2]
+  B_V_FULL = 16,      // [2]
+  B_V_EMPTY = 18,     // [2]
+  B_S_FULL = 20,      // [2][2]
+  B_S_FREE = 24,      // [2][2]
+  B_P_FULL = 28,      // [2]
+  B_P_EMPTY = 30      // [2]
 };
 
-// TMEM columns: S^T buffers at 0 and 64, O^T at 128.
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0, kColO = 128;
+// TMEM columns per stream: two S^T buffers and the O^T accumulator.
+constexpr uint32_t kTmemCols = 512;
+__device__ __forceinline__ uint32_t col_s(int stream, uint32_t buf) { return stream * 192 + buf * 64; }
+__device__ __forceinline__ uint32_t col_o(int stream) { return stream * 192 + 128; }
 
 struct ItemSlot {
   int b, h, i, n, diag_last;
@@ -133,10 +159,10 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 
 // Bounded wait. Returns false (and raises the CTA abort flag and the device
 // error) when the phase does not complete within the limit, or at once when
-// the CTA is already aborting.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                       WsHeader* hdr, int where) {
-  if (mbar_try(bar, parity)) return true;
+// the CTA is already aborting. The first probe is inlined; the spin loop is
+// out of line so that callers keep their registers on the fast path.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                            WsHeader* hdr, int where) {
   const unsigned long long t0 = now_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
@@ -149,6 +175,12 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          WsHeader* hdr, int where) {
+  if (mbar_try(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, hdr, where);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
@@ -240,17 +272,20 @@ __device__ __forceinline__ void add_bf16_pair(float& lo, float& hi, uint32_t w) 
   hi += __uint_as_float(w & 0xffff0000u);
 }
 
-// Named barrier over the 128 softmax threads (id 1), optionally OR-reducing a predicate.
-__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-__device__ __forceinline__ bool softmax_any(bool pred) {
+// Named barrier over the 128 threads of one softmax warpgroup (id 1 + stream),
+// optionally OR-reducing a predicate.
+__device__ __forceinline__ void softmax_sync(int id) {
+  asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+}
+__device__ __forceinline__ bool softmax_any(int id, bool pred) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "setp.ne.u32 p, %2, 0;\n\t"
+      "bar.red.or.pred q, %1, 128, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)pred)
+      : "r"(id), "r"((uint32_t)pred)
       : "memory");
   return r != 0;
 }
@@ -306,6 +341,71 @@ __device__ __forceinline__ void decode_item(const TcArgs& a, int item, int& b, i
   h = kvh * a.group + rem % a.group;
 }
 
+// Two per-stream values kept in registers (a runtime-indexed array would live
+// in local memory).
+template <class T>
+struct Pair {
+  T v0, v1;
+  __device__ __forceinline__ T get(int x) const { return x ? v1 : v0; }
+  __device__ __forceinline__ void set(int x, T v) {
+    if (x) v1 = v;
+    else v0 = v;
+  }
+  __device__ __forceinline__ T inc(int x) {  // post-increment
+    const T old = get(x);
+    set(x, old + 1);
+    return old;
+  }
+};
+
+// The (stream, chunk) walk shared by the producer and both MMA issuers.
+// Streams alternate one chunk at a time; a stream whose item has no chunks
+// moves on to its next item without taking a step; once one stream runs out
+// of items the other takes every remaining step.
+struct Walk {
+  Pair<int> t;     // item counter of the stream (slot = t & 1)
+  Pair<int> c;     // next chunk of the current item
+  Pair<int> C;     // chunks of the current item; -1: no item open
+  Pair<int> done;
+  int turn;
+  __device__ __forceinline__ void init() {
+    t = {0, 0};
+    c = {0, 0};
+    C = {-1, -1};
+    done = {0, 0};
+    turn = 0;
+  }
+  // Chooses the stream of the next step; -1 when both are finished.
+  __device__ __forceinline__ int pick() const {
+    int x = turn;
+    if (done.get(x)) x ^= 1;
+    return done.get(x) ? -1 : x;
+  }
+  // Opens an item of n kept blocks on stream x (n = 0: closed at once).
+  __device__ __forceinline__ void open(int x, int n) {
+    const int chunks = (n + 1) >> 1;
+    c.set(x, 0);
+    if (chunks == 0) {
+      C.set(x, -1);
+      t.inc(x);
+    } else {
+      C.set(x, chunks);
+    }
+  }
+  // After a step of stream x: advance, and close the item after its last chunk.
+  __device__ __forceinline__ void advance(int x) {
+    turn = x ^ 1;
+    const int nc = c.get(x) + 1;
+    if (nc == C.get(x)) {
+      c.set(x, 0);
+      C.set(x, -1);
+      t.inc(x);
+    } else {
+      c.set(x, nc);
+    }
+  }
+};
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, TcArgs a) {
@@ -313,32 +413,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  int* sList = reinterpret_cast<int*>(smem + kOffList);
-  float* sRed = reinterpret_cast<float*>(smem + kOffRed);
-  float* sM = reinterpret_cast<float*>(smem + kOffM);
-  float* sL = reinterpret_cast<float*>(smem + kOffL);
-  float* sA = reinterpret_cast<float*>(smem + kOffA);
   const uint32_t bars = sbase + kOffBar;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-  ItemSlot* sItem = reinterpret_cast<ItemSlot*>(smem + kOffMisc + 16);  // 2 slots
+  ItemSlot* sItem = reinterpret_cast<ItemSlot*>(smem + kOffMisc + 16);  // [stream][slot]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   auto bar = [&](int idx) { return bars + 8u * idx; };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(B_ITEM_FULL + s), 1);
-      mbar_init(bar(B_ITEM_EMPTY + s), 2);
-      mbar_init(bar(B_Q_FULL + s), 1);
-      mbar_init(bar(B_Q_EMPTY + s), 1);
-      mbar_init(bar(B_K_FULL + s), 1);
-      mbar_init(bar(B_K_EMPTY + s), 1);
-      mbar_init(bar(B_V_FULL + s), 1);
-      mbar_init(bar(B_V_EMPTY + s), 1);
-      mbar_init(bar(B_S_FULL + s), 1);
-      mbar_init(bar(B_P_FULL + s), 128);
-      mbar_init(bar(B_P_EMPTY + s), 1);
+    for (int x = 0; x < kStreams; ++x) {
+      for (int u = 0; u < 2; ++u) {
+        mbar_init(bar(B_ITEM_FULL + 2 * x + u), 1);
+        mbar_init(bar(B_ITEM_EMPTY + 2 * x + u), 4);
+        mbar_init(bar(B_S_FULL + 2 * x + u), 1);
+        mbar_init(bar(B_S_FREE + 2 * x + u), 128);
+      }
+      mbar_init(bar(B_Q_FULL + x), 1);
+      mbar_init(bar(B_Q_EMPTY + x), 1);
+      mbar_init(bar(B_P_FULL + x), 128);
+      mbar_init(bar(B_P_EMPTY + x), 1);
+      mbar_init(bar(B_K_FULL + x), 1);
+      mbar_init(bar(B_K_EMPTY + x), 1);
+      mbar_init(bar(B_V_FULL + x), 1);
+      mbar_init(bar(B_V_EMPTY + x), 1);
     }
     *sAbort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -356,293 +454,425 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = *sTmem;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ producer
-    uint32_t gq = 0, gk = 0, gv = 0;
-    // per ring: bit 2u set = stage u has an issued load, bit u = that load's phase parity
-    uint32_t lastQ = 0, lastK = 0, lastV = 0;
-    for (int t = 0;; ++t) {
-      const int s = t & 1;
+  if (warp < 4) {
+    if (warp == 0) {
+      // ---------------------------------------------------------------- K producer
+      // Fetches work items, compacts their kept lists into the item slot,
+      // publishes them, and loads the Q tiles and the K tiles.
+      int16_t* const lists = reinterpret_cast<int16_t*>(smem + kOffList);
+      uint32_t gk = 0;
+      Pair<uint32_t> gq = {0u, 0u};
+      Pair<uint32_t> gs = {0u, 0u};  // S^T uses per stream, as counted by the S issuer
+      // per K stage u: bit 8u: loaded once; bits 8u+1..: s_full barrier index and
+      // parity of the S^T step that read it (the stage is free once that completes)
+      uint32_t kuse = 0;
+      // bit u set: ring stage u has an issued load; bit 2+u: its phase parity
+      uint32_t lastK = 0, lastQ = 0;
+      Pair<int> kvrow = {0, 0};
+      Pair<int> nkept = {0, 0};
       bool ok = true;
-      if (lane == 0 && t >= 2) ok = mbar_wait(bar(B_ITEM_EMPTY + s), ((t >> 1) - 1) & 1, sAbort, a.hdr, 1);
-      int item = 0;
-      if (lane == 0) item = (*sAbort) ? a.n_items : (int)atomicAdd(&a.hdr->work[0], 1u);
-      item = __shfl_sync(0xffffffffu, item, 0);
-      if (item >= a.n_items) {
-        if (lane == 0) {
-          sItem[s].n = -1;
-          mbar_arrive(bar(B_ITEM_FULL + s));
-        }
-        break;
-      }
-      int b, h, i;
-      decode_item(a, item, b, h, i);
-      const size_t row_id = ((size_t)b * a.Hq + h) * a.nb + i;
-      int n_raw = a.cnt[row_id];
-      if (n_raw < 0 || n_raw > a.W) {
-        if (lane == 0) raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnTc, (int)row_id, n_raw);
-        n_raw = n_raw < 0 ? 0 : a.W;
-      }
-      const int32_t* lst = a.idx + row_id * a.W;
-      int n = 0;
-      for (int base = 0; base < n_raw; base += 32) {
-        const int t2 = base + lane;
-        int j = t2 < n_raw ? lst[t2] : -1;
-        const bool in = t2 < n_raw;
-        const bool valid = in && j >= 0 && j <= i;
-        if (in && !valid) raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnTc, (int)row_id, j);
-        const uint32_t m = __ballot_sync(0xffffffffu, valid);
-        if (valid) sList[n + __popc(m & ((1u << lane) - 1u))] = j;
-        n += __popc(m);
-      }
-      __syncwarp();
-      if (lane == 0) {
-        sItem[s].b = b;
-        sItem[s].h = h;
-        sItem[s].i = i;
-        sItem[s].n = n;
-        sItem[s].diag_last = (n > 0 && sList[n - 1] == i) ? 1 : 0;
-        mbar_arrive(bar(B_ITEM_FULL + s));
-        if (n > 0 && ok) {
-          const uint32_t qb = gq & 1;
-          if (gq >= 2) ok = mbar_wait(bar(B_Q_EMPTY + qb), ((gq >> 1) - 1) & 1, sAbort, a.hdr, 2);
-          const int qrow = (int)(((size_t)b * a.Hq + h) * a.N + (size_t)i * kBS);
-          if (ok) {
-            mbar_expect_tx(bar(B_Q_FULL + qb), kQBytes);
-            const uint32_t dq = sbase + kOffQ + qb * kQBytes;
-            tma_load_2d(dq, &tmQ, 0, qrow, bar(B_Q_FULL + qb));
-            tma_load_2d(dq + kQBytes / 2, &tmQ, 64, qrow, bar(B_Q_FULL + qb));
-            lastQ = (lastQ & ~(5u << qb)) | (4u << qb) | (((gq >> 1) & 1u) << qb);
+      Walk wk;
+      wk.init();
+      for (;;) {
+        const int x = wk.pick();
+        if (x < 0) break;
+        if (wk.C.get(x) < 0) {
+          // open the stream's next item: fetch it, compact its list, publish it
+          const int tx = wk.t.get(x);
+          const int slot = tx & 1;
+          if (lane == 0 && tx >= 2)
+            ok = ok && mbar_wait(bar(B_ITEM_EMPTY + 2 * x + slot), ((tx >> 1) - 1) & 1, sAbort, a.hdr, 1);
+          int item = 0;
+          if (lane == 0) item = (!ok || *sAbort) ? a.n_items : (int)atomicAdd(&a.hdr->work[0], 1u);
+          item = __shfl_sync(0xffffffffu, item, 0);
+          if (item >= a.n_items) {
+            if (lane == 0) {
+              sItem[2 * x + slot].n = -1;
+              mbar_arrive(bar(B_ITEM_FULL + 2 * x + slot));
+            }
+            wk.done.set(x, 1);
+            continue;
           }
-          ++gq;
-          const int kvrow0 = (int)(((size_t)b * a.Hkv + h / a.group) * a.N);
-          const int C = (n + 1) >> 1;
-          for (int c = 0; c < C && ok; ++c) {
-            const int nblk = min(2, n - 2 * c);
-            const uint32_t ks = gk & 1;
-            if (gk >= 2) ok = mbar_wait(bar(B_K_EMPTY + ks), ((gk >> 1) - 1) & 1, sAbort, a.hdr, 3);
-            if (!ok) break;
+          int b, h, i;
+          decode_item(a, item, b, h, i);
+          const size_t row_id = ((size_t)b * a.Hq + h) * a.nb + i;
+          int n_raw = a.cnt[row_id];
+          if (n_raw < 0 || n_raw > a.W) {
+            if (lane == 0) raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnTc, (int)row_id, n_raw);
+            n_raw = n_raw < 0 ? 0 : a.W;
+          }
+          const int32_t* lst = a.idx + row_id * a.W;
+          int16_t* my_list = lists + (2 * x + slot) * kMaxBlocks;
+          int n = 0;
+          for (int base = 0; base < n_raw; base += 32) {
+            const int t2 = base + lane;
+            const bool in = t2 < n_raw;
+            const int j = in ? lst[t2] : -1;
+            const bool valid = in && j >= 0 && j <= i;
+            if (in && !valid) raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnTc, (int)row_id, j);
+            const uint32_t m = __ballot_sync(0xffffffffu, valid);
+            if (valid) my_list[n + __popc(m & ((1u << lane) - 1u))] = (int16_t)j;
+            n += __popc(m);
+          }
+          __syncwarp();
+          if (lane == 0) {
+            ItemSlot& sl = sItem[2 * x + slot];
+            sl.b = b;
+            sl.h = h;
+            sl.i = i;
+            sl.n = n;
+            sl.diag_last = (n > 0 && my_list[n - 1] == i) ? 1 : 0;
+            mbar_arrive(bar(B_ITEM_FULL + 2 * x + slot));
+            if (n > 0) {
+              const uint32_t gqx = gq.get(x);
+              if (gqx >= 1) ok = ok && mbar_wait(bar(B_Q_EMPTY + x), (gqx - 1) & 1, sAbort, a.hdr, 2);
+              if (ok) {
+                const int qrow = (int)(((size_t)b * a.Hq + h) * a.N + (size_t)i * kBS);
+                mbar_expect_tx(bar(B_Q_FULL + x), kQBytes);
+                const uint32_t dq = sbase + kOffQ + x * kQBytes;
+                tma_load_2d(dq, &tmQ, 0, qrow, bar(B_Q_FULL + x));
+                tma_load_2d(dq + kQBytes / 2, &tmQ, 64, qrow, bar(B_Q_FULL + x));
+                lastQ = (lastQ & ~(5u << x)) | (1u << x) | ((gqx & 1u) << (2 + x));
+              }
+              gq.inc(x);
+            }
+          }
+          __syncwarp();
+          kvrow.set(x, (int)(((size_t)b * a.Hkv + h / a.group) * a.N));
+          nkept.set(x, n);
+          wk.open(x, n);
+          continue;
+        }
+        // one step: the K tile of chunk c of stream x
+        if (lane == 0 && ok) {
+          const int c = wk.c.get(x);
+          const int nblk = min(2, nkept.get(x) - 2 * c);
+          const int kvr = kvrow.get(x);
+          const int16_t* my_list = lists + (2 * x + (wk.t.get(x) & 1)) * kMaxBlocks;
+          const uint32_t ks = gk & 1;
+          const uint32_t prev = (kuse >> (8 * ks)) & 0xffu;
+          if (prev & 1u) ok = ok && mbar_wait(bar(B_S_FULL + (prev >> 2)), (prev >> 1) & 1u, sAbort, a.hdr, 3);
+          if (ok) {
             mbar_expect_tx(bar(B_K_FULL + ks), nblk * (kKVBytes / 2));
             const uint32_t dk = sbase + kOffK + ks * kKVBytes;
             for (int bb = 0; bb < nblk; ++bb) {
-              const int row = kvrow0 + sList[2 * c + bb] * kBS;
+              const int row = kvr + my_list[2 * c + bb] * kBS;
               tma_load_2d(dk + bb * (kKVBytes / 4), &tmK, 0, row, bar(B_K_FULL + ks));
               tma_load_2d(dk + kKVBytes / 2 + bb * (kKVBytes / 4), &tmK, 64, row, bar(B_K_FULL + ks));
             }
-            lastK = (lastK & ~(5u << ks)) | (4u << ks) | (((gk >> 1) & 1u) << ks);
-            ++gk;
-            const uint32_t vs = gv & 1;
-            if (gv >= 2) ok = mbar_wait(bar(B_V_EMPTY + vs), ((gv >> 1) - 1) & 1, sAbort, a.hdr, 4);
-            if (!ok) break;
+            lastK = (lastK & ~(5u << ks)) | (1u << ks) | (((gk >> 1) & 1u) << (2 + ks));
+          }
+          // the S^T step of this K tile writes buffer gs & 1 of stream x
+          const uint32_t gsx = gs.get(x);
+          const uint32_t use = 1u | (((gsx >> 1) & 1u) << 1) | ((uint32_t)(2 * x + (gsx & 1)) << 2);
+          kuse = (kuse & ~(0xffu << (8 * ks))) | (use << (8 * ks));
+        }
+        gs.inc(x);
+        ++gk;
+        ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+        wk.advance(x);
+      }
+      // drain: every issued load has landed before the CTA may exit
+      if (lane == 0) {
+        volatile int no_abort = 0;
+        for (int u = 0; u < 2; ++u) {
+          if (lastK & (1u << u)) mbar_wait(bar(B_K_FULL + u), (lastK >> (2 + u)) & 1u, &no_abort, a.hdr, 5);
+          if (lastQ & (1u << u)) mbar_wait(bar(B_Q_FULL + u), (lastQ >> (2 + u)) & 1u, &no_abort, a.hdr, 5);
+        }
+      }
+    } else if (warp == 3) {
+      // ---------------------------------------------------------------- V producer
+      // Walks the same steps; reads each item's kept list from its slot and
+      // releases the slot after the item's last V tile has been issued.
+      const int16_t* const lists = reinterpret_cast<const int16_t*>(smem + kOffList);
+      if (lane == 0) {
+        uint32_t gv = 0;
+        uint32_t lastV = 0;
+        Pair<int> kvrow = {0, 0};
+        Pair<int> nkept = {0, 0};
+        bool ok = true;
+        Walk wk;
+        wk.init();
+        for (;;) {
+          const int x = wk.pick();
+          if (x < 0) break;
+          if (wk.C.get(x) < 0) {
+            const int tx = wk.t.get(x);
+            const int slot = tx & 1;
+            ok = ok && mbar_wait(bar(B_ITEM_FULL + 2 * x + slot), (tx >> 1) & 1, sAbort, a.hdr, 6);
+            const ItemSlot it = sItem[2 * x + slot];
+            const int n = ok ? it.n : -1;
+            if (n <= 0) mbar_arrive(bar(B_ITEM_EMPTY + 2 * x + slot));
+            if (n < 0) {
+              wk.done.set(x, 1);
+              continue;
+            }
+            kvrow.set(x, (int)(((size_t)it.b * a.Hkv + it.h / a.group) * a.N));
+            nkept.set(x, n);
+            wk.open(x, n);
+            continue;
+          }
+          const int c = wk.c.get(x);
+          const int slot = wk.t.get(x) & 1;
+          const int nblk = min(2, nkept.get(x) - 2 * c);
+          const uint32_t vs = gv & 1;
+          if (gv >= 2) ok = ok && mbar_wait(bar(B_V_EMPTY + vs), ((gv >> 1) - 1) & 1, sAbort, a.hdr, 4);
+          if (ok) {
+            const int16_t* my_list = lists + (2 * x + slot) * kMaxBlocks;
+            const int kvr = kvrow.get(x);
             mbar_expect_tx(bar(B_V_FULL + vs), nblk * (kKVBytes / 2));
             const uint32_t dv = sbase + kOffV + vs * kKVBytes;
             for (int bb = 0; bb < nblk; ++bb) {
-              const int row = kvrow0 + sList[2 * c + bb] * kBS;
+              const int row = kvr + my_list[2 * c + bb] * kBS;
               tma_load_2d(dv + bb * (kKVBytes / 4), &tmV, 0, row, bar(B_V_FULL + vs));
               tma_load_2d(dv + kKVBytes / 2 + bb * (kKVBytes / 4), &tmV, 64, row, bar(B_V_FULL + vs));
             }
-            lastV = (lastV & ~(5u << vs)) | (4u << vs) | (((gv >> 1) & 1u) << vs);
-            ++gv;
+            lastV = (lastV & ~(5u << vs)) | (1u << vs) | (((gv >> 1) & 1u) << (2 + vs));
           }
+          ++gv;
+          if (c == wk.C.get(x) - 1) mbar_arrive(bar(B_ITEM_EMPTY + 2 * x + slot));
+          wk.advance(x);
         }
+        volatile int no_abort = 0;
+        for (int u = 0; u < 2; ++u)
+          if (lastV & (1u << u)) mbar_wait(bar(B_V_FULL + u), (lastV >> (2 + u)) & 1u, &no_abort, a.hdr, 5);
       }
-      __syncwarp();
-    }
-    // drain: every issued load has landed before the CTA may exit
-    if (lane == 0) {
-      volatile int no_abort = 0;
-      for (int u = 0; u < 2; ++u) {
-        if (lastK & (4u << u)) mbar_wait(bar(B_K_FULL + u), (lastK >> u) & 1u, &no_abort, a.hdr, 5);
-        if (lastV & (4u << u)) mbar_wait(bar(B_V_FULL + u), (lastV >> u) & 1u, &no_abort, a.hdr, 5);
-        if (lastQ & (4u << u)) mbar_wait(bar(B_Q_FULL + u), (lastQ >> u) & 1u, &no_abort, a.hdr, 5);
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t gq = 0, gk = 0, gv = 0, gs = 0, gp = 0;
-      bool ok = true;
-      auto issue_pv = [&](int c, int n) {
-        const uint32_t pb = gp & 1, vs = gv & 1;
-        ok = ok && mbar_wait(bar(B_P_FULL + pb), (gp >> 1) & 1, sAbort, a.hdr, 10);
-        ok = ok && mbar_wait(bar(B_V_FULL + vs), (gv >> 1) & 1, sAbort, a.hdr, 11);
-        tc_fence_after();
-        if (ok) {
-          const int ksteps = min(2, n - 2 * c) * (kBS / 16);
-          const uint32_t va = sbase + kOffV + vs * kKVBytes;
-          const uint32_t pa = sbase + kOffP + pb * kPBytes;
-          for (int kk = 0; kk < ksteps; ++kk) {
-            const uint64_t adesc = smem_desc(va + kk * 2048, kKVBytes / 2, 1024);
-            const uint64_t bdesc = smem_desc(pa + kk * 2048, kPBytes, 1024);
-            tc_mma(tmem + kColO, adesc, bdesc, kIdescPV, (c > 0 || kk > 0) ? 1u : 0u);
-          }
-        }
-        tc_commit(bar(B_P_EMPTY + pb));
-        tc_commit(bar(B_V_EMPTY + vs));
-        ++gp;
-        ++gv;
-      };
-      for (int t = 0;; ++t) {
-        const int s = t & 1;
-        if (!mbar_wait(bar(B_ITEM_FULL + s), (t >> 1) & 1, sAbort, a.hdr, 12)) break;
-        const int n = sItem[s].n;
-        mbar_arrive(bar(B_ITEM_EMPTY + s));
-        if (n < 0) break;
-        if (n == 0) continue;
-        const int C = (n + 1) >> 1;
-        const uint32_t qb = gq & 1;
-        ok = ok && mbar_wait(bar(B_Q_FULL + qb), (gq >> 1) & 1, sAbort, a.hdr, 13);
-        for (int c = 0; c < C; ++c) {
-          const uint32_t ks = gk & 1, sb = gs & 1;
-          ok = ok && mbar_wait(bar(B_K_FULL + ks), (gk >> 1) & 1, sAbort, a.hdr, 14);
-          tc_fence_after();
-          if (ok) {
-            const uint32_t ka = sbase + kOffK + ks * kKVBytes;
-            const uint32_t qa = sbase + kOffQ + qb * kQBytes;
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint64_t adesc = smem_desc(ka + (kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32, 16, 1024);
-              const uint64_t bdesc = smem_desc(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024);
-              tc_mma(tmem + kColS + sb * kBS, adesc, bdesc, kIdescS, kk > 0 ? 1u : 0u);
+    } else if (warp == 1 || warp == 2) {
+      // ---------------------------------------------------------------- MMA issuers
+      const bool is_s = warp == 1;
+      if (lane == 0) {
+        uint32_t gk = 0, gv = 0;
+        Pair<uint32_t> gs = {0u, 0u};   // S^T uses per stream (buffer = gs & 1)
+        Pair<uint32_t> gq = {0u, 0u};   // Q tiles per stream
+        Pair<uint32_t> gp = {0u, 0u};   // P tiles per stream
+        Pair<int> nkept = {0, 0};
+        bool ok = true;
+        Walk wk;
+        wk.init();
+        // descriptor templates: k-steps only advance the 14-bit start-address field
+        const uint64_t dK0 = smem_desc(sbase + kOffK, 16, 1024);
+        const uint64_t dQ0 = smem_desc(sbase + kOffQ, 16, 1024);
+        const uint64_t dV0 = smem_desc(sbase + kOffV, kKVBytes / 2, 1024);
+        const uint64_t dP0 = smem_desc(sbase + kOffP, kPBytes, 1024);
+        for (;;) {
+          const int x = wk.pick();
+          if (x < 0) break;
+          if (wk.C.get(x) < 0) {
+            const int tx = wk.t.get(x);
+            const int slot = tx & 1;
+            ok = ok && mbar_wait(bar(B_ITEM_FULL + 2 * x + slot), (tx >> 1) & 1, sAbort, a.hdr, 12);
+            const int n = ok ? sItem[2 * x + slot].n : -1;
+            mbar_arrive(bar(B_ITEM_EMPTY + 2 * x + slot));
+            if (n < 0) {
+              wk.done.set(x, 1);
+              continue;
             }
+            nkept.set(x, n);
+            wk.open(x, n);
+            if (n > 0 && is_s) ok = ok && mbar_wait(bar(B_Q_FULL + x), gq.inc(x) & 1, sAbort, a.hdr, 13);
+            continue;
           }
-          tc_commit(bar(B_S_FULL + sb));
-          tc_commit(bar(B_K_EMPTY + ks));
-          if (c == C - 1) tc_commit(bar(B_Q_EMPTY + qb));
-          ++gk;
-          ++gs;
-          if (c >= 1) issue_pv(c - 1, n);
+          const int c = wk.c.get(x);
+          if (is_s) {
+            const uint32_t gsx = gs.get(x);
+            const uint32_t ks = gk & 1, sb = gsx & 1;
+            ok = ok && mbar_wait(bar(B_K_FULL + ks), (gk >> 1) & 1, sAbort, a.hdr, 14);
+            if (gsx >= 2)
+              ok = ok && mbar_wait(bar(B_S_FREE + 2 * x + sb), ((gsx >> 1) - 1) & 1, sAbort, a.hdr, 15);
+            tc_fence_after();
+            if (ok) {
+              const uint64_t dk = dK0 + (uint64_t)((ks * kKVBytes) >> 4);
+              const uint64_t dq = dQ0 + (uint64_t)((x * kQBytes) >> 4);
+              const uint32_t d = tmem + col_s(x, sb);
+#pragma unroll
+              for (int kk = 0; kk < kD / 16; ++kk)
+                tc_mma(d, dk + (uint64_t)(((kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32) >> 4),
+                       dq + (uint64_t)(((kk >> 2) * (kQBytes / 2) + (kk & 3) * 32) >> 4), kIdescS,
+                       kk > 0 ? 1u : 0u);
+            }
+            tc_commit(bar(B_S_FULL + 2 * x + sb));  // also frees K stage ks
+            if (c == wk.C.get(x) - 1) tc_commit(bar(B_Q_EMPTY + x));
+            ++gk;
+            gs.inc(x);
+          } else {
+            const uint32_t vs = gv & 1;
+            ok = ok && mbar_wait(bar(B_P_FULL + x), gp.get(x) & 1, sAbort, a.hdr, 10);
+            ok = ok && mbar_wait(bar(B_V_FULL + vs), (gv >> 1) & 1, sAbort, a.hdr, 11);
+            tc_fence_after();
+            if (ok) {
+              const int ksteps = min(2, nkept.get(x) - 2 * c) * (kBS / 16);
+              const uint64_t dv = dV0 + (uint64_t)((vs * kKVBytes) >> 4);
+              const uint64_t dp = dP0 + (uint64_t)((x * kPBytes) >> 4);
+              const uint32_t d = tmem + col_o(x);
+              for (int kk = 0; kk < ksteps; ++kk)
+                tc_mma(d, dv + (uint64_t)(kk * 128), dp + (uint64_t)(kk * 128), kIdescPV,
+                       (c > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(bar(B_P_EMPTY + x));
+            tc_commit(bar(B_V_EMPTY + vs));
+            ++gv;
+            gp.inc(x);
+          }
+          wk.advance(x);
         }
-        issue_pv(C - 1, n);
-        ++gq;
+        // the tensor core has finished every MMA before TMEM is released
+        volatile int no_abort = 0;
+        for (int x = 0; x < kStreams; ++x) {
+          const uint32_t np = gp.get(x), ns = gs.get(x);
+          if (!is_s && np > 0) mbar_wait(bar(B_P_EMPTY + x), (np - 1) & 1, &no_abort, a.hdr, 16);
+          if (is_s && ns > 0)
+            mbar_wait(bar(B_S_FULL + 2 * x + ((ns - 1) & 1)), ((ns - 1) >> 1) & 1, &no_abort, a.hdr, 17);
+        }
       }
-      // wait for the last MMAs before TMEM is released
-      volatile int no_abort = 0;
-      if (gp > 0) mbar_wait(bar(B_P_EMPTY + ((gp - 1) & 1)), ((gp - 1) >> 1) & 1, &no_abort, a.hdr, 15);
     }
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    const int sp = warp - 4;            // TMEM sub-partition: lanes 32*sp ..
-    const int r = sp * 32 + lane;       // key row of S^T / head-dim row of O^T
+    const int x = (warp - 4) / 4;        // stream
+    const int sp = warp & 3;             // TMEM sub-partition: lanes 32*sp ..
+    const int r = sp * 32 + lane;        // key row of S^T / head-dim row of O^T
+    const int bar_id = 1 + x;
     const uint32_t lane_addr = (uint32_t)(sp * 32) << 16;
     const float c2 = a.scale_log2;
-    float l[64];  // this thread's share of the row sums (running maxima live in sM)
+    float* const sRed = reinterpret_cast<float*>(smem + kOffRed) + x * 256;
+    float* const sM = reinterpret_cast<float*>(smem + kOffM) + x * 64;
+    float* const sL = reinterpret_cast<float*>(smem + kOffL) + x * 64;
+    float* const sA = reinterpret_cast<float*>(smem + kOffA) + x * 64;
+    float* const sT = reinterpret_cast<float*>(smem + kOffT) + x * 64;
+    uint8_t* const pbuf = smem + kOffP + x * kPBytes;
+    float l[64];  // this thread's share of the row sums
     uint32_t gs = 0, gp = 0;
-    uint32_t pend = 0, ph_empty = 0;  // bit b: P buffer b awaits its PV / parity of its next phase
-    auto wait_pv = [&](uint32_t pb) {
-      if (pend & (1u << pb)) {
-        mbar_wait(bar(B_P_EMPTY + pb), (ph_empty >> pb) & 1u, sAbort, a.hdr, 20);
-        ph_empty ^= 1u << pb;
-        pend &= ~(1u << pb);
+    bool pend = false;  // a PV of this stream's P tile has not been waited for
+    auto wait_pv = [&]() {
+      if (pend) {
+        mbar_wait(bar(B_P_EMPTY + x), (gp - 1) & 1, sAbort, a.hdr, 20);
+        pend = false;
       }
     };
     for (int t = 0;; ++t) {
-      const int s = t & 1;
-      mbar_wait(bar(B_ITEM_FULL + s), (t >> 1) & 1, sAbort, a.hdr, 21);
-      const ItemSlot it = sItem[s];
+      const int slot = t & 1;
+      mbar_wait(bar(B_ITEM_FULL + 2 * x + slot), (t >> 1) & 1, sAbort, a.hdr, 21);
+      const ItemSlot it = sItem[2 * x + slot];
       // one decision for the whole warpgroup (also orders the slot reads before the release)
-      const bool stop = softmax_any(it.n < 0 || *sAbort != 0);
-      if (threadIdx.x == 128) mbar_arrive(bar(B_ITEM_EMPTY + s));
+      const bool stop = softmax_any(bar_id, it.n < 0 || *sAbort != 0);
+      if (r == 0) mbar_arrive(bar(B_ITEM_EMPTY + 2 * x + slot));
       if (stop) break;
       const int C = (it.n + 1) >> 1;
 #pragma unroll
       for (int q = 0; q < 64; ++q) l[q] = 0.f;
       for (int c = 0; c < C; ++c) {
         const uint32_t sb = gs & 1;
-        const uint32_t s_addr = tmem + lane_addr + kColS + sb * kBS;
-        mbar_wait(bar(B_S_FULL + sb), (gs >> 1) & 1, sAbort, a.hdr, 22);
-        ++gs;
+        mbar_wait(bar(B_S_FULL + 2 * x + sb), (gs >> 1) & 1, sAbort, a.hdr, 22);
         tc_fence_after();
         const int nblk = min(2, it.n - 2 * c);
         const int blk = r / kBS, kl = r % kBS;
-        const bool valid = blk < nblk;
+        const bool valid = blk < nblk;  // this lane holds a kept key of the tile
         const bool diag = (c == C - 1) && it.diag_last && (blk == nblk - 1);
-        float x[64];
-        auto load_logits = [&]() {
-          uint32_t raw[64];
-          tmem_ld64(s_addr, raw);
-#pragma unroll
-          for (int q = 0; q < 64; ++q) {
-            float v = __uint_as_float(raw[q]) * c2;
-            if (!valid || (diag && kl > q)) v = -INFINITY;
-            x[q] = v;
-          }
-        };
-        load_logits();
-        // the first tile sets the maxima; later tiles raise them only past the threshold
-        bool raise = (c == 0);
-        if (!raise) {
-          float dmax = -INFINITY;
+        const uint32_t s_addr = tmem + lane_addr + col_s(x, sb);
+        uint32_t raw[64];
+        tmem_ld64(s_addr, raw);
+        // Raise the running maxima when some visible logit exceeds them by more
+        // than 2^kTau, tested as S > (m + kTau) / scale; the first tile sets them.
+        bool big = false;
+        if (c > 0 && valid) {
+          bool part[8] = {false, false, false, false, false, false, false, false};
 #pragma unroll
           for (int q4 = 0; q4 < 16; ++q4) {
-            const float4 mv = reinterpret_cast<const float4*>(sM)[q4];
-            dmax = fmaxf(dmax, fmaxf(fmaxf(x[4 * q4] - mv.x, x[4 * q4 + 1] - mv.y),
-                                     fmaxf(x[4 * q4 + 2] - mv.z, x[4 * q4 + 3] - mv.w)));
+            const float4 tv = reinterpret_cast<const float4*>(sT)[q4];
+            const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int q = 4 * q4 + e;
+              part[q & 7] |= (__uint_as_float(raw[q]) > tt[e]) && !(diag && kl > q);
+            }
           }
-          raise = softmax_any(dmax > kTau);
+          big = ((part[0] | part[1]) | (part[2] | part[3])) | ((part[4] | part[5]) | (part[6] | part[7]));
         }
-        if (raise) {
-          const int col0 = warp_col_reduce<true>(x, lane);
-          sRed[sp * 64 + col0] = x[0];
-          sRed[sp * 64 + col0 + 1] = x[1];
-          softmax_sync();
+        if (c == 0 || softmax_any(bar_id, big)) {
+          // column maxima of d = S * scale - m over this tile's visible keys
+#pragma unroll
+          for (int q4 = 0; q4 < 16; ++q4) {
+            const float4 mv = c == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : reinterpret_cast<const float4*>(sM)[q4];
+            const float mm[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int q = 4 * q4 + e;
+              const bool vis = valid && !(diag && kl > q);
+              raw[q] = __float_as_uint(vis ? __fmaf_rn(__uint_as_float(raw[q]), c2, -mm[e]) : -INFINITY);
+            }
+          }
+          float* dv = reinterpret_cast<float*>(raw);
+          const int col0 = warp_col_reduce<true>(*reinterpret_cast<float(*)[64]>(dv), lane);
+          sRed[sp * 64 + col0] = dv[0];
+          sRed[sp * 64 + col0 + 1] = dv[1];
+          softmax_sync(bar_id);
           if (r < 64) {
             const float mx = fmaxf(fmaxf(sRed[r], sRed[64 + r]), fmaxf(sRed[128 + r], sRed[192 + r]));
-            const float mo = sM[r];
-            const float mn = (c == 0) ? mx : fmaxf(mo, mx);
-            sA[r] = (c == 0) ? 0.f : ex2(mo - mn);
+            const float inc = c == 0 ? mx : fmaxf(mx, 0.f);
+            const float mn = c == 0 ? mx : sM[r] + inc;
+            sA[r] = inc;
             sM[r] = mn;
+            sT[r] = c2 > 0.f ? (mn + kTau) / c2 : INFINITY;
           }
-          softmax_sync();
+          softmax_sync(bar_id);
           if (c > 0) {
             // O^T must hold every earlier tile's contribution before it is rescaled
-            wait_pv(0);
-            wait_pv(1);
+            wait_pv();
             tc_fence_after();
-            uint32_t o[64];
-            tmem_ld64(tmem + lane_addr + kColO, o);
+            tmem_ld64(tmem + lane_addr + col_o(x), raw);
 #pragma unroll
             for (int q = 0; q < 64; ++q) {
-              const float alpha = sA[q];
+              const float alpha = ex2(-sA[q]);
               l[q] *= alpha;
-              o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+              raw[q] = __float_as_uint(__uint_as_float(raw[q]) * alpha);
             }
-            tmem_st64(tmem + lane_addr + kColO, o);
+            tmem_st64(tmem + lane_addr + col_o(x), raw);
           }
-          load_logits();
+          tmem_ld64(s_addr, raw);  // the tile again, for the exponentials
         }
-        // P = 2^(x - m) in bf16, row r of the MN-major P^T tile
-        const uint32_t pb = gp & 1;
-        wait_pv(pb);
-        uint8_t* prow = smem + kOffP + pb * kPBytes + r * 128;
+        tc_fence_before();
+        mbar_arrive(bar(B_S_FREE + 2 * x + sb));  // the S^T buffer may be refilled
+        ++gs;
+        // P = 2^(S * scale - m) in bf16, row r of the MN-major P^T tile; the row
+        // sums add the same bf16 values
+        wait_pv();
+        uint8_t* const prow = pbuf + r * 128;
+        if (!valid) {
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          float p[8];
-          const float4 m0 = reinterpret_cast<const float4*>(sM)[2 * cc];
-          const float4 m1 = reinterpret_cast<const float4*>(sM)[2 * cc + 1];
-          const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+          for (int cc = 0; cc < 8; ++cc)
+            *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        } else {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) p[e] = ex2(x[cc * 8 + e] - mm[e]);
-          uint4 w;
-          w.x = pack_bf16(p[0], p[1]);
-          w.y = pack_bf16(p[2], p[3]);
-          w.z = pack_bf16(p[4], p[5]);
-          w.w = pack_bf16(p[6], p[7]);
-          // row sums of the bf16 values the tensor core multiplies
-          add_bf16_pair(l[cc * 8 + 0], l[cc * 8 + 1], w.x);
-          add_bf16_pair(l[cc * 8 + 2], l[cc * 8 + 3], w.y);
-          add_bf16_pair(l[cc * 8 + 4], l[cc * 8 + 5], w.z);
-          add_bf16_pair(l[cc * 8 + 6], l[cc * 8 + 7], w.w);
-          *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = w;
+          for (int cc = 0; cc < 8; ++cc) {
+            const float4 m0 = reinterpret_cast<const float4*>(sM)[2 * cc];
+            const float4 m1 = reinterpret_cast<const float4*>(sM)[2 * cc + 1];
+            const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+            float pv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int q = cc * 8 + e;
+              const float dq = __fmaf_rn(__uint_as_float(raw[q]), c2, -mm[e]);
+              pv[e] = (diag && kl > q) ? 0.f : ex2(dq);
+            }
+            uint4 w;
+            w.x = pack_bf16(pv[0], pv[1]);
+            w.y = pack_bf16(pv[2], pv[3]);
+            w.z = pack_bf16(pv[4], pv[5]);
+            w.w = pack_bf16(pv[6], pv[7]);
+            add_bf16_pair(l[cc * 8 + 0], l[cc * 8 + 1], w.x);
+            add_bf16_pair(l[cc * 8 + 2], l[cc * 8 + 3], w.y);
+            add_bf16_pair(l[cc * 8 + 4], l[cc * 8 + 5], w.z);
+            add_bf16_pair(l[cc * 8 + 6], l[cc * 8 + 7], w.w);
+            *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = w;
+          }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
-        mbar_arrive(bar(B_P_FULL + pb));
-        pend |= 1u << pb;
+        mbar_arrive(bar(B_P_FULL + x));
+        pend = true;
         ++gp;
       }
       // ---------------------------------------------------------------- epilogue
-      wait_pv(0);
-      wait_pv(1);
+      wait_pv();
       tc_fence_after();
       warp_col_reduce<false>(l, lane);
       {
@@ -651,39 +881,39 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         sRed[sp * 64 + col0] = l[0];
         sRed[sp * 64 + col0 + 1] = l[1];
       }
-      softmax_sync();
-      if (r < 64) sL[r] = (sRed[r] + sRed[64 + r]) + (sRed[128 + r] + sRed[192 + r]);
-      softmax_sync();
+      softmax_sync(bar_id);
+      float lsum = 0.f;
+      if (r < 64) {
+        lsum = (sRed[r] + sRed[64 + r]) + (sRed[128 + r] + sRed[192 + r]);
+        sL[r] = lsum > 0.f ? 1.0f / lsum : 0.f;
+      }
+      softmax_sync(bar_id);
       const size_t row0 = ((size_t)it.b * a.Hq + it.h) * a.N + (size_t)it.i * kBS;
-      uint8_t* stage = smem + kOffP;  // both P buffers are idle here
       {
         uint32_t o[64];
         if (C > 0) {
-          tmem_ld64(tmem + lane_addr + kColO, o);
+          tmem_ld64(tmem + lane_addr + col_o(x), o);
         } else {
 #pragma unroll
           for (int q = 0; q < 64; ++q) o[q] = 0u;
         }
         tc_fence_before();
+        // the P tile is idle here: stage O (row q, column r) in it
 #pragma unroll
-        for (int q = 0; q < 64; ++q) {
-          const float lq = sL[q];
-          const float v = lq > 0.f ? __uint_as_float(o[q]) / lq : 0.f;
-          reinterpret_cast<__nv_bfloat16*>(stage)[q * kD + r] = __float2bfloat16_rn(v);
-        }
+        for (int q = 0; q < 64; ++q)
+          reinterpret_cast<__nv_bfloat16*>(pbuf)[q * kD + r] =
+              __float2bfloat16_rn(__uint_as_float(o[q]) * sL[q]);
       }
-      softmax_sync();
+      softmax_sync(bar_id);
       {
-        const uint4* src = reinterpret_cast<const uint4*>(stage);
+        const uint4* src = reinterpret_cast<const uint4*>(pbuf);
         uint4* dst = reinterpret_cast<uint4*>(a.out + row0 * kD);
 #pragma unroll
         for (int e = 0; e < (kBS * kD / 8) / 128; ++e) dst[e * 128 + r] = src[e * 128 + r];
       }
-      if (a.lse != nullptr && r < 64) {
-        const float lq = sL[r];
-        a.lse[row0 + r] = (C > 0 && lq > 0.f) ? (sM[r] * kLn2 + logf(lq)) : -INFINITY;
-      }
-      softmax_sync();
+      if (a.lse != nullptr && r < 64)
+        a.lse[row0 + r] = (C > 0 && lsum > 0.f) ? (sM[r] * kLn2 + logf(lsum)) : -INFINITY;
+      softmax_sync(bar_id);
     }
   }
 
