@@ -73,11 +73,10 @@ constexpr int kOffV = kOffK + 2 * kKVBytes;               // 2 ring stages
 constexpr int kOffP = kOffV + 2 * kKVBytes;               // one per stream
 constexpr int kOffList = kOffP + kStreams * kPBytes;      // [stream][slot][kMaxBlocks] int16
 constexpr int kOffRed = kOffList + kStreams * 2 * kMaxBlocks * 2;  // [stream][4][64] f32
-constexpr int kOffM = kOffRed + kStreams * 4 * 64 * 4;    // [stream][64] running max
+constexpr int kOffM = kOffRed + kStreams * 4 * 64 * 4;    // [stream][64] -(running max)
 constexpr int kOffL = kOffM + kStreams * 64 * 4;          // [stream][64] 1 / row sum
 constexpr int kOffA = kOffL + kStreams * 64 * 4;          // [stream][64] max increments
-constexpr int kOffT = kOffA + kStreams * 64 * 4;          // [stream][64] raise thresholds on S
-constexpr int kOffBar = kOffT + kStreams * 64 * 4;        // mbarriers
+constexpr int kOffBar = kOffA + kStreams * 64 * 4;        // mbarriers
 constexpr int kNumBars = 32;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;          // tmem base, abort flag, item slots
 constexpr int kSmemBytes = kOffMisc + 128 + 1024;         // + alignment slack
@@ -734,12 +733,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t lane_addr = (uint32_t)(sp * 32) << 16;
     const float c2 = a.scale_log2;
     float* const sRed = reinterpret_cast<float*>(smem + kOffRed) + x * 256;
-    float* const sM = reinterpret_cast<float*>(smem + kOffM) + x * 64;
+    float* const sNM = reinterpret_cast<float*>(smem + kOffM) + x * 64;  // -(running max)
     float* const sL = reinterpret_cast<float*>(smem + kOffL) + x * 64;
     float* const sA = reinterpret_cast<float*>(smem + kOffA) + x * 64;
-    float* const sT = reinterpret_cast<float*>(smem + kOffT) + x * 64;
     uint8_t* const pbuf = smem + kOffP + x * kPBytes;
-    float l[64];  // this thread's share of the row sums
+    float2 l2[32];  // this thread's share of the row sums, queries 2j and 2j+1
+    float tmin = INFINITY;  // smallest (m + kTau) / scale over the queries
     uint32_t gs = 0, gp = 0;
     bool pend = false;  // a PV of this stream's P tile has not been waited for
     auto wait_pv = [&]() {
@@ -758,7 +757,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (stop) break;
       const int C = (it.n + 1) >> 1;
 #pragma unroll
-      for (int q = 0; q < 64; ++q) l[q] = 0.f;
+      for (int q2 = 0; q2 < 32; ++q2) l2[q2] = make_float2(0.f, 0.f);
       for (int c = 0; c < C; ++c) {
         const uint32_t sb = gs & 1;
         mbar_wait(bar(B_S_FULL + 2 * x + sb), (gs >> 1) & 1, sAbort, a.hdr, 22);
@@ -771,33 +770,50 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         uint32_t raw[64];
         tmem_ld64(s_addr, raw);
         // Raise the running maxima when some visible logit exceeds them by more
-        // than 2^kTau, tested as S > (m + kTau) / scale; the first tile sets them.
-        bool big = false;
-        if (c > 0 && valid) {
-          bool part[8] = {false, false, false, false, false, false, false, false};
+        // than 2^kTau. Cheap sufficient test first: no S value of this lane
+        // above the smallest per-query threshold (m + kTau) / scale.
+        bool raise = c == 0;
+        if (!raise) {
+          float mx = -INFINITY;
+          if (valid) {
+            float t8[8];
 #pragma unroll
-          for (int q4 = 0; q4 < 16; ++q4) {
-            const float4 tv = reinterpret_cast<const float4*>(sT)[q4];
-            const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
+            for (int e = 0; e < 8; ++e) t8[e] = __uint_as_float(raw[e]);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int q = 4 * q4 + e;
-              part[q & 7] |= (__uint_as_float(raw[q]) > tt[e]) && !(diag && kl > q);
-            }
+            for (int q = 8; q < 64; ++q) t8[q & 7] = fmaxf(t8[q & 7], __uint_as_float(raw[q]));
+            mx = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
+                       fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
           }
-          big = ((part[0] | part[1]) | (part[2] | part[3])) | ((part[4] | part[5]) | (part[6] | part[7]));
+          if (softmax_any(bar_id, mx > tmin)) {
+            // exact test, query by query
+            bool part[8] = {false, false, false, false, false, false, false, false};
+            if (valid) {
+#pragma unroll
+              for (int q4 = 0; q4 < 16; ++q4) {
+                const float4 nm = reinterpret_cast<const float4*>(sNM)[q4];
+                const float mm[4] = {nm.x, nm.y, nm.z, nm.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int q = 4 * q4 + e;
+                  part[q & 7] |= (__fmaf_rn(__uint_as_float(raw[q]), c2, mm[e]) > kTau) && !(diag && kl > q);
+                }
+              }
+            }
+            const bool big = ((part[0] | part[1]) | (part[2] | part[3])) | ((part[4] | part[5]) | (part[6] | part[7]));
+            raise = softmax_any(bar_id, big);
+          }
         }
-        if (c == 0 || softmax_any(bar_id, big)) {
+        if (raise) {
           // column maxima of d = S * scale - m over this tile's visible keys
 #pragma unroll
           for (int q4 = 0; q4 < 16; ++q4) {
-            const float4 mv = c == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : reinterpret_cast<const float4*>(sM)[q4];
-            const float mm[4] = {mv.x, mv.y, mv.z, mv.w};
+            const float4 nm = c == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : reinterpret_cast<const float4*>(sNM)[q4];
+            const float mm[4] = {nm.x, nm.y, nm.z, nm.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int q = 4 * q4 + e;
               const bool vis = valid && !(diag && kl > q);
-              raw[q] = __float_as_uint(vis ? __fmaf_rn(__uint_as_float(raw[q]), c2, -mm[e]) : -INFINITY);
+              raw[q] = __float_as_uint(vis ? __fmaf_rn(__uint_as_float(raw[q]), c2, mm[e]) : -INFINITY);
             }
           }
           float* dv = reinterpret_cast<float*>(raw);
@@ -808,22 +824,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (r < 64) {
             const float mx = fmaxf(fmaxf(sRed[r], sRed[64 + r]), fmaxf(sRed[128 + r], sRed[192 + r]));
             const float inc = c == 0 ? mx : fmaxf(mx, 0.f);
-            const float mn = c == 0 ? mx : sM[r] + inc;
             sA[r] = inc;
-            sM[r] = mn;
-            sT[r] = c2 > 0.f ? (mn + kTau) / c2 : INFINITY;
+            sNM[r] = c == 0 ? -mx : sNM[r] - inc;
           }
           softmax_sync(bar_id);
+          // smallest raise threshold of the new maxima
+          {
+            float mn = INFINITY;
+#pragma unroll
+            for (int q4 = 0; q4 < 16; ++q4) {
+              const float4 nm = reinterpret_cast<const float4*>(sNM)[q4];
+              mn = fminf(mn, fminf(fminf(-nm.x, -nm.y), fminf(-nm.z, -nm.w)));
+            }
+            tmin = c2 > 0.f ? (mn + kTau) / c2 : INFINITY;
+          }
           if (c > 0) {
             // O^T must hold every earlier tile's contribution before it is rescaled
             wait_pv();
             tc_fence_after();
             tmem_ld64(tmem + lane_addr + col_o(x), raw);
 #pragma unroll
-            for (int q = 0; q < 64; ++q) {
-              const float alpha = ex2(-sA[q]);
-              l[q] *= alpha;
-              raw[q] = __float_as_uint(__uint_as_float(raw[q]) * alpha);
+            for (int q2 = 0; q2 < 32; ++q2) {
+              const float2 al = make_float2(ex2(-sA[2 * q2]), ex2(-sA[2 * q2 + 1]));
+              l2[q2] = __fmul2_rn(l2[q2], al);
+              const float2 o = __fmul2_rn(make_float2(__uint_as_float(raw[2 * q2]), __uint_as_float(raw[2 * q2 + 1])), al);
+              raw[2 * q2] = __float_as_uint(o.x);
+              raw[2 * q2 + 1] = __float_as_uint(o.y);
             }
             tmem_st64(tmem + lane_addr + col_o(x), raw);
           }
@@ -841,28 +867,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int cc = 0; cc < 8; ++cc)
             *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
         } else {
+          const float2 c22 = make_float2(c2, c2);
 #pragma unroll
           for (int cc = 0; cc < 8; ++cc) {
-            const float4 m0 = reinterpret_cast<const float4*>(sM)[2 * cc];
-            const float4 m1 = reinterpret_cast<const float4*>(sM)[2 * cc + 1];
-            const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-            float pv[8];
+            const float4 n0 = reinterpret_cast<const float4*>(sNM)[2 * cc];
+            const float4 n1 = reinterpret_cast<const float4*>(sNM)[2 * cc + 1];
+            const float2 nm[4] = {make_float2(n0.x, n0.y), make_float2(n0.z, n0.w), make_float2(n1.x, n1.y),
+                                  make_float2(n1.z, n1.w)};
+            uint32_t w[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int q = cc * 8 + e;
-              const float dq = __fmaf_rn(__uint_as_float(raw[q]), c2, -mm[e]);
-              pv[e] = (diag && kl > q) ? 0.f : ex2(dq);
+            for (int e = 0; e < 4; ++e) {
+              const int q = cc * 8 + 2 * e;
+              const float2 d2 = __ffma2_rn(make_float2(__uint_as_float(raw[q]), __uint_as_float(raw[q + 1])), c22, nm[e]);
+              float p0 = ex2(d2.x), p1 = ex2(d2.y);
+              if (diag) {
+                p0 = kl > q ? 0.f : p0;
+                p1 = kl > q + 1 ? 0.f : p1;
+              }
+              w[e] = pack_bf16(p0, p1);
+              l2[q >> 1] = __fadd2_rn(l2[q >> 1], make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u)));
             }
-            uint4 w;
-            w.x = pack_bf16(pv[0], pv[1]);
-            w.y = pack_bf16(pv[2], pv[3]);
-            w.z = pack_bf16(pv[4], pv[5]);
-            w.w = pack_bf16(pv[6], pv[7]);
-            add_bf16_pair(l[cc * 8 + 0], l[cc * 8 + 1], w.x);
-            add_bf16_pair(l[cc * 8 + 2], l[cc * 8 + 3], w.y);
-            add_bf16_pair(l[cc * 8 + 4], l[cc * 8 + 5], w.z);
-            add_bf16_pair(l[cc * 8 + 6], l[cc * 8 + 7], w.w);
-            *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = w;
+            *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -874,12 +899,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // ---------------------------------------------------------------- epilogue
       wait_pv();
       tc_fence_after();
-      warp_col_reduce<false>(l, lane);
       {
-        const int col0 = ((lane >> 4) & 1) * 32 + ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 +
-                         ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
-        sRed[sp * 64 + col0] = l[0];
-        sRed[sp * 64 + col0 + 1] = l[1];
+        float* lf = reinterpret_cast<float*>(l2);
+        const int col0 = warp_col_reduce<false>(*reinterpret_cast<float(*)[64]>(lf), lane);
+        sRed[sp * 64 + col0] = lf[0];
+        sRed[sp * 64 + col0 + 1] = lf[1];
       }
       softmax_sync(bar_id);
       float lsum = 0.f;
@@ -912,7 +936,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int e = 0; e < (kBS * kD / 8) / 128; ++e) dst[e * 128 + r] = src[e * 128 + r];
       }
       if (a.lse != nullptr && r < 64)
-        a.lse[row0 + r] = (C > 0 && lsum > 0.f) ? (sM[r] * kLn2 + logf(lsum)) : -INFINITY;
+        a.lse[row0 + r] = (C > 0 && lsum > 0.f) ? (-sNM[r] * kLn2 + logf(lsum)) : -INFINITY;
       softmax_sync(bar_id);
     }
   }
