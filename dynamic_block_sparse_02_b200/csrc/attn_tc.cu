@@ -70,15 +70,16 @@ constexpr int kPBytes = kChunk * kBS * 2;     // 16 KB: [128 keys][64 queries] b
 constexpr int kOffQ = 0;                                  // one per stream
 constexpr int kOffK = kOffQ + kStreams * kQBytes;         // 2 ring stages
 constexpr int kOffV = kOffK + 2 * kKVBytes;               // 2 ring stages
-constexpr int kOffP = kOffV + 2 * kKVBytes;               // one per stream
-constexpr int kOffList = kOffP + kStreams * kPBytes;      // [stream][slot][kMaxBlocks] int16
+constexpr int kPTiles = 3;                                // P tiles shared by the streams
+constexpr int kOffP = kOffV + 2 * kKVBytes;               // [kPTiles]
+constexpr int kOffList = kOffP + kPTiles * kPBytes;       // [stream][slot][kMaxBlocks] int16
 constexpr int kOffRed = kOffList + kStreams * 2 * kMaxBlocks * 2;  // [stream][4][64] f32
 constexpr int kOffM = kOffRed + kStreams * 4 * 64 * 4;    // [stream][64] -(running max)
 constexpr int kOffL = kOffM + kStreams * 64 * 4;          // [stream][64] 1 / row sum
 constexpr int kOffA = kOffL + kStreams * 64 * 4;          // [stream][64] max increments
 constexpr int kOffBar = kOffA + kStreams * 64 * 4;        // mbarriers
-constexpr int kNumBars = 32;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;          // tmem base, abort flag, item slots
+constexpr int kNumBars = 36;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;          // tmem base, abort flag, item slots, step ids
 constexpr int kSmemBytes = kOffMisc + 128 + 1024;         // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -94,9 +95,14 @@ enum {
   B_V_EMPTY = 18,     // [2]
   B_S_FULL = 20,      // [2][2]
   B_S_FREE = 24,      // [2][2]
-  B_P_FULL = 28,      // [2]
-  B_P_EMPTY = 30      // [2]
+  B_P_FULL = 28,      // [kPTiles]
+  B_P_EMPTY = 31,     // [kPTiles]
+  B_O_DONE = 34       // [2]: the last PV of a stream's item has finished
 };
+
+// P tiles: step n of the (stream, chunk) walk writes tile n % kPTiles, whose
+// previous reader was step n - kPTiles; the S^T issuer publishes each step's
+// index next to its S^T buffer (sStep[stream][buffer]).
 
 // TMEM columns per stream: two S^T buffers and the O^T accumulator.
 constexpr uint32_t kTmemCols = 512;
@@ -416,6 +422,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   ItemSlot* sItem = reinterpret_cast<ItemSlot*>(smem + kOffMisc + 16);  // [stream][slot]
+  volatile uint32_t* sStep = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc + 112);  // [stream][S buffer]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   auto bar = [&](int idx) { return bars + 8u * idx; };
@@ -425,17 +432,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int u = 0; u < 2; ++u) {
         mbar_init(bar(B_ITEM_FULL + 2 * x + u), 1);
         mbar_init(bar(B_ITEM_EMPTY + 2 * x + u), 4);
-        mbar_init(bar(B_S_FULL + 2 * x + u), 1);
+        mbar_init(bar(B_S_FULL + 2 * x + u), 2);  // MMA commit + step-id publication
         mbar_init(bar(B_S_FREE + 2 * x + u), 128);
       }
       mbar_init(bar(B_Q_FULL + x), 1);
       mbar_init(bar(B_Q_EMPTY + x), 1);
-      mbar_init(bar(B_P_FULL + x), 128);
-      mbar_init(bar(B_P_EMPTY + x), 1);
+      mbar_init(bar(B_O_DONE + x), 1);
       mbar_init(bar(B_K_FULL + x), 1);
       mbar_init(bar(B_K_EMPTY + x), 1);
       mbar_init(bar(B_V_FULL + x), 1);
       mbar_init(bar(B_V_EMPTY + x), 1);
+    }
+    for (int t = 0; t < kPTiles; ++t) {
+      mbar_init(bar(B_P_FULL + t), 128);
+      mbar_init(bar(B_P_EMPTY + t), 1);
     }
     *sAbort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -689,26 +699,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                        dq + (uint64_t)(((kk >> 2) * (kQBytes / 2) + (kk & 3) * 32) >> 4), kIdescS,
                        kk > 0 ? 1u : 0u);
             }
+            sStep[2 * x + sb] = gk;
             tc_commit(bar(B_S_FULL + 2 * x + sb));  // also frees K stage ks
+            mbar_arrive(bar(B_S_FULL + 2 * x + sb));  // releases the step id
             if (c == wk.C.get(x) - 1) tc_commit(bar(B_Q_EMPTY + x));
             ++gk;
             gs.inc(x);
           } else {
             const uint32_t vs = gv & 1;
-            ok = ok && mbar_wait(bar(B_P_FULL + x), gp.get(x) & 1, sAbort, a.hdr, 10);
+            const uint32_t pt = gv % kPTiles, pu = gv / kPTiles;
+            ok = ok && mbar_wait(bar(B_P_FULL + pt), pu & 1, sAbort, a.hdr, 10);
             ok = ok && mbar_wait(bar(B_V_FULL + vs), (gv >> 1) & 1, sAbort, a.hdr, 11);
             tc_fence_after();
             if (ok) {
               const int ksteps = min(2, nkept.get(x) - 2 * c) * (kBS / 16);
               const uint64_t dv = dV0 + (uint64_t)((vs * kKVBytes) >> 4);
-              const uint64_t dp = dP0 + (uint64_t)((x * kPBytes) >> 4);
+              const uint64_t dp = dP0 + (uint64_t)((pt * kPBytes) >> 4);
               const uint32_t d = tmem + col_o(x);
               for (int kk = 0; kk < ksteps; ++kk)
                 tc_mma(d, dv + (uint64_t)(kk * 128), dp + (uint64_t)(kk * 128), kIdescPV,
                        (c > 0 || kk > 0) ? 1u : 0u);
             }
-            tc_commit(bar(B_P_EMPTY + x));
+            tc_commit(bar(B_P_EMPTY + pt));
             tc_commit(bar(B_V_EMPTY + vs));
+            if (c == wk.C.get(x) - 1) tc_commit(bar(B_O_DONE + x));
             ++gv;
             gp.inc(x);
           }
@@ -716,9 +730,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         // the tensor core has finished every MMA before TMEM is released
         volatile int no_abort = 0;
+        if (!is_s && gv > 0)
+          mbar_wait(bar(B_P_EMPTY + (gv - 1) % kPTiles), ((gv - 1) / kPTiles) & 1, &no_abort, a.hdr, 16);
         for (int x = 0; x < kStreams; ++x) {
-          const uint32_t np = gp.get(x), ns = gs.get(x);
-          if (!is_s && np > 0) mbar_wait(bar(B_P_EMPTY + x), (np - 1) & 1, &no_abort, a.hdr, 16);
+          const uint32_t ns = gs.get(x);
           if (is_s && ns > 0)
             mbar_wait(bar(B_S_FULL + 2 * x + ((ns - 1) & 1)), ((ns - 1) >> 1) & 1, &no_abort, a.hdr, 17);
         }
@@ -736,16 +751,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     float* const sNM = reinterpret_cast<float*>(smem + kOffM) + x * 64;  // -(running max)
     float* const sL = reinterpret_cast<float*>(smem + kOffL) + x * 64;
     float* const sA = reinterpret_cast<float*>(smem + kOffA) + x * 64;
-    uint8_t* const pbuf = smem + kOffP + x * kPBytes;
     float2 l2[32];  // this thread's share of the row sums, queries 2j and 2j+1
     float tmin = INFINITY;  // smallest (m + kTau) / scale over the queries
-    uint32_t gs = 0, gp = 0;
-    bool pend = false;  // a PV of this stream's P tile has not been waited for
-    auto wait_pv = [&]() {
-      if (pend) {
-        mbar_wait(bar(B_P_EMPTY + x), (gp - 1) & 1, sAbort, a.hdr, 20);
-        pend = false;
-      }
+    uint32_t gs = 0;
+    uint32_t go = 0;      // items of this stream whose O^T has been completed
+    uint32_t lastn = 0;   // walk step of this stream's previous tile
+    // wait until the PV of walk step n has finished
+    auto wait_step_pv = [&](uint32_t n) {
+      mbar_wait(bar(B_P_EMPTY + n % kPTiles), (n / kPTiles) & 1, sAbort, a.hdr, 20);
     };
     for (int t = 0;; ++t) {
       const int slot = t & 1;
@@ -762,6 +775,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const uint32_t sb = gs & 1;
         mbar_wait(bar(B_S_FULL + 2 * x + sb), (gs >> 1) & 1, sAbort, a.hdr, 22);
         tc_fence_after();
+        const uint32_t n_step = sStep[2 * x + sb];  // this tile's walk step
         const int nblk = min(2, it.n - 2 * c);
         const int blk = r / kBS, kl = r % kBS;
         const bool valid = blk < nblk;  // this lane holds a kept key of the tile
@@ -840,7 +854,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           if (c > 0) {
             // O^T must hold every earlier tile's contribution before it is rescaled
-            wait_pv();
+            wait_step_pv(lastn);
             tc_fence_after();
             tmem_ld64(tmem + lane_addr + col_o(x), raw);
 #pragma unroll
@@ -859,9 +873,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mbar_arrive(bar(B_S_FREE + 2 * x + sb));  // the S^T buffer may be refilled
         ++gs;
         // P = 2^(S * scale - m) in bf16, row r of the MN-major P^T tile; the row
-        // sums add the same bf16 values
-        wait_pv();
-        uint8_t* const prow = pbuf + r * 128;
+        // sums add the same bf16 values. The tile was last read by step n - kPTiles.
+        if (n_step >= (uint32_t)kPTiles) wait_step_pv(n_step - kPTiles);
+        uint8_t* const prow = smem + kOffP + (n_step % kPTiles) * kPBytes + r * 128;
         if (!valid) {
 #pragma unroll
           for (int cc = 0; cc < 8; ++cc)
@@ -892,12 +906,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
-        mbar_arrive(bar(B_P_FULL + x));
-        pend = true;
-        ++gp;
+        mbar_arrive(bar(B_P_FULL + n_step % kPTiles));
+        lastn = n_step;
       }
       // ---------------------------------------------------------------- epilogue
-      wait_pv();
+      if (C > 0) {
+        // the item's last PV has finished: O^T is complete
+        mbar_wait(bar(B_O_DONE + x), go & 1, sAbort, a.hdr, 23);
+        ++go;
+      }
       tc_fence_after();
       {
         float* lf = reinterpret_cast<float*>(l2);
@@ -922,18 +939,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int q = 0; q < 64; ++q) o[q] = 0u;
         }
         tc_fence_before();
-        // the P tile is idle here: stage O (row q, column r) in it
+        // thread r holds column r of the 64 output rows: each warp store covers
+        // 32 consecutive head-dim elements of one row
+        __nv_bfloat16* const dst = a.out + row0 * kD + r;
 #pragma unroll
-        for (int q = 0; q < 64; ++q)
-          reinterpret_cast<__nv_bfloat16*>(pbuf)[q * kD + r] =
-              __float2bfloat16_rn(__uint_as_float(o[q]) * sL[q]);
-      }
-      softmax_sync(bar_id);
-      {
-        const uint4* src = reinterpret_cast<const uint4*>(pbuf);
-        uint4* dst = reinterpret_cast<uint4*>(a.out + row0 * kD);
-#pragma unroll
-        for (int e = 0; e < (kBS * kD / 8) / 128; ++e) dst[e * 128 + r] = src[e * 128 + r];
+        for (int q = 0; q < 64; ++q) dst[(size_t)q * kD] = __float2bfloat16_rn(__uint_as_float(o[q]) * sL[q]);
       }
       if (a.lse != nullptr && r < 64)
         a.lse[row0 + r] = (C > 0 && lsum > 0.f) ? (-sNM[r] * kLn2 + logf(lsum)) : -INFINITY;
