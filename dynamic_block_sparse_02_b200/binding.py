@@ -54,6 +54,7 @@ SIGNATURES = {
     "dsa_block_scores": (ctypes.c_int, [_P, _vp, _vp, _f32p, _vp, _sz, _vp]),
     "dsa_topk_select": (ctypes.c_int, [_P, _f32p, _i32p, _i32p, _vp]),
     "dsa_select_blocks": (ctypes.c_int, [_P, _vp, _vp, _i32p, _i32p, _vp, _sz, _vp]),
+    "dsa_select_blocks_static": (ctypes.c_int, [_P, _vp, _vp, _i32p, _i32p, _vp]),
     "dsa_sparse_attn_fwd": (ctypes.c_int, [_P, _vp, _vp, _vp, _i32p, _i32p, _vp, _f32p, _vp, _sz, _vp]),
     "dsa_forward": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _f32p, _i32p, _i32p, _vp, _sz, _vp]),
     "dsa_check_status": (ctypes.c_int, [_vp, _vp]),
@@ -162,6 +163,11 @@ def dsa_topk_select(p: Params, scores, idx, cnt, stream=None) -> None:
 def dsa_select_blocks(p: Params, q, k, idx, cnt, ws, ws_bytes: int, stream=None) -> None:
     _check(_lib.dsa_select_blocks(p.ref, _ptr(q), _ptr(k), _ptr(idx), _ptr(cnt), _ptr(ws),
                                   ws_bytes, _stream(stream)), "dsa_select_blocks")
+
+
+def dsa_select_blocks_static(p: Params, q, k, idx, cnt, stream=None) -> None:
+    _check(_lib.dsa_select_blocks_static(p.ref, _ptr(q), _ptr(k), _ptr(idx), _ptr(cnt),
+                                         _stream(stream)), "dsa_select_blocks_static")
 
 
 def dsa_sparse_attn_fwd(p: Params, q, k, v, idx, cnt, out, lse, ws, ws_bytes: int,

@@ -4,6 +4,7 @@
 // purpose to read the device error flag.
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "dsa_internal.cuh"
 
@@ -151,6 +152,63 @@ dsa_status run_selection(const dsa_params* p, const Shape& s, const dsa_bf16* q,
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Selection with its scratch in static device memory (dsa_select_blocks_static).
+//
+// Some callers cannot hand the library a workspace: a plain C host program
+// that runs the selection step inside a loop where it may not allocate device
+// memory, because cudaMalloc/cudaFree can synchronise the whole device and
+// stall work queued by others, or a runtime that plans all device memory once
+// at start-up and has no spare region for this step. For them the pooled
+// blocks Qp and Kp live in this file-scope array instead of a workspace. The
+// array belongs to this library's module: the CUDA driver places it in device
+// memory when it loads the module on a device, and this code never allocates.
+//
+// Limit: Qp and Kp together (each rounded up to 256 bytes) must fit in
+// kStaticScratchBytes = 16 MiB, which holds e.g. B=1, Hq=32, Hkv=8, N=32768,
+// block=64, d=128 (8 MiB + 2 MiB). Larger problems get DSA_ERR_WORKSPACE.
+//
+// Nothing in the array has to start at zero: the pooling kernel writes every
+// pooled value before the score/select kernel reads it. There is one array per
+// device (per process), so two calls that overlap on one device (two streams,
+// two host threads) race on it and must be ordered by the caller.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+
+static __device__ __align__(256) unsigned char g_select_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {nullptr};
+
+// Device address of g_select_scratch on the current device. The first call on
+// a device looks it up with cudaGetSymbolAddress (which may load the module on
+// that device); later calls return the cached address.
+dsa_status select_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_select_scratch) != cudaSuccess || addr == nullptr)
+      return DSA_ERR_CUDA;
+    g_scratch_addr[dev] = addr;
+  }
+  *out = g_scratch_addr[dev];
+  return DSA_OK;
+}
+
+// Bytes of g_select_scratch one problem needs: Qp then Kp.
+size_t static_scratch_need(const Shape& s, size_t* kp_off) {
+  *kp_off = round_up((size_t)s.B * s.Hq * s.nb * s.d * sizeof(float));
+  return *kp_off + round_up((size_t)s.B * s.Hkv * s.nb * s.d * sizeof(float));
+}
+
+}  // namespace
+
 extern "C" {
 
 size_t dsa_kmax(const dsa_params* p) {
@@ -219,6 +277,32 @@ dsa_status dsa_select_blocks(const dsa_params* p, const dsa_bf16* q, const dsa_b
   if ((st = check_ws(s, ws, ws_bytes)) != DSA_OK) return st;
   if ((st = check_device()) != DSA_OK) return st;
   return run_selection(p, s, q, k, idx, cnt, ws, (cudaStream_t)stream);
+}
+
+dsa_status dsa_select_blocks_static(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k,
+                                    int32_t* idx, int32_t* cnt, void* stream) {
+  Shape s;
+  dsa_status st = make_shape(p, &s);
+  if (st != DSA_OK) return st;
+  if (is_empty(p)) return DSA_OK;
+  if (q == nullptr || k == nullptr || (idx == nullptr && s.W > 0) || cnt == nullptr ||
+      !aligned16(q) || !aligned16(k))
+    return DSA_ERR_INVALID_ARG;
+  size_t kp_off = 0;
+  if (static_scratch_need(s, &kp_off) > kStaticScratchBytes) return DSA_ERR_WORKSPACE;
+  if ((st = check_device()) != DSA_OK) return st;
+  void* scratch = nullptr;
+  if ((st = select_scratch(&scratch)) != DSA_OK) return st;
+  char* base = static_cast<char*>(scratch);
+  float* qp = reinterpret_cast<float*>(base);
+  float* kp = reinterpret_cast<float*>(base + kp_off);
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = dsa::launch_pool(s, reinterpret_cast<const __nv_bfloat16*>(q),
+                                   reinterpret_cast<const __nv_bfloat16*>(k), qp, kp, cs);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  // No workspace header here: the selection kernel's row-overflow guard still
+  // skips an out-of-range write but has no flag to set.
+  return from_cuda(dsa::launch_score_select(s, budgets(p), qp, kp, idx, cnt, nullptr, cs));
 }
 
 dsa_status dsa_sparse_attn_fwd(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k,

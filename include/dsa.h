@@ -32,7 +32,9 @@
  *     padded with -1; cnt int32 [B, Hq, nb] holds each row's length. When
  *     W == 0 (no block can be kept) idx may be NULL.
  *   - The caller owns all memory. The library never allocates device or host
- *     memory; it uses the caller's workspace (dsa_workspace_size bytes).
+ *     memory; it uses the caller's workspace (dsa_workspace_size bytes), except
+ *     dsa_select_blocks_static, whose scratch is the library's static device
+ *     array.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream) and do not synchronise the host, so a sequence of calls
  *     can be captured into a CUDA graph.
@@ -41,7 +43,8 @@
  *     bounded wait that gave up) set a flag in the workspace header; read it
  *     with dsa_check_status.
  *   - The device must be an sm_100a GPU (B200). The library holds no state
- *     except, per device, a cache of the kernels' shared-memory attributes.
+ *     except, per device, a cache of the kernels' shared-memory attributes
+ *     and the static scratch array of dsa_select_blocks_static.
  */
 #ifndef DSA_H
 #define DSA_H
@@ -137,6 +140,31 @@ dsa_status dsa_topk_select(const dsa_params *p, const float *scores, int32_t *id
 dsa_status dsa_select_blocks(const dsa_params *p, const dsa_bf16 *q, const dsa_bf16 *k,
                              int32_t *idx, int32_t *cnt, void *ws, size_t ws_bytes,
                              void *stream);
+
+/*
+ * Steps 1-3 like dsa_select_blocks, for callers that cannot give the library
+ * a workspace (a host loop that may not call cudaMalloc, which can
+ * synchronise the device; a runtime whose device memory is planned once at
+ * start-up). The pages describe no such variant: it exists only so that the
+ * selection can run with no caller memory besides q, k, idx and cnt.
+ *   - Scratch: the pooled blocks live in a 16 MiB array in the library's own
+ *     static device memory (one per device, placed there when the CUDA driver
+ *     loads the library's module); nothing is allocated and nothing in it
+ *     needs to start at zero. A problem whose pooled Qp and Kp (fp32,
+ *     B*(Hq+Hkv)*nb*d*4 bytes, each part rounded up to 256) exceed 16 MiB gets
+ *     DSA_ERR_WORKSPACE and launches nothing.
+ *   - Set-up: the first call on a device looks the array's address up
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture on the device.
+ *   - Overlapping calls on one device (two streams, two host threads) share
+ *     the array and race: order them (one stream, or events).
+ *   - Arguments, outputs and argument errors as dsa_select_blocks; the result
+ *     equals dsa_select_blocks bit for bit. There is no workspace header, so
+ *     no device error flag is set (the selection kernel still skips any write
+ *     past a row's W entries).
+ */
+dsa_status dsa_select_blocks_static(const dsa_params *p, const dsa_bf16 *q, const dsa_bf16 *k,
+                                    int32_t *idx, int32_t *cnt, void *stream);
 
 /*
  * Step 4 on a caller selection. idx/cnt as above, W = dsa_kmax(p); every
