@@ -80,7 +80,7 @@ constexpr int kOffA = kOffL + kStreams * 64 * 4;          // [stream][64] max in
 constexpr int kOffBar = kOffA + kStreams * 64 * 4;        // mbarriers
 constexpr int kNumBars = 36;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;          // tmem base, abort flag, item slots, step ids
-constexpr int kSmemBytes = kOffMisc + 128 + 1024;         // + alignment slack
+constexpr int kSmemBytes = kOffMisc + 160 + 1024;         // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // barrier indices ([stream] or [stream][slot|buffer] or [stage])
@@ -186,6 +186,39 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                                           WsHeader* hdr, int where) {
   if (mbar_try(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, abort_flag, hdr, where);
+}
+
+// Step metadata word: stream, first and last chunk of the item, kept blocks in the chunk.
+__device__ __forceinline__ uint32_t step_meta(int x, bool first, bool last, int nblk) {
+  return (uint32_t)x | (first ? 2u : 0u) | (last ? 4u : 0u) | ((uint32_t)nblk << 3);
+}
+
+// Waits for a barrier phase that belongs to walk step n. Returns 1 when the
+// phase completed, 0 when the walk has fewer than n + 1 steps (the step and
+// its phase never come), -1 when the kernel is aborting or the wait timed out.
+__device__ __noinline__ int step_wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* total,
+                                           uint32_t n, volatile int* abort_flag, WsHeader* hdr,
+                                           int where) {
+  const unsigned long long t0 = now_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return 1;
+    if (*total <= n) return 0;
+    if ((it & 63u) == 0u) {
+      if (*abort_flag) return -1;
+      if (now_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        raise_error(hdr, DSA_ERR_DEVICE_TIMEOUT, kKernAttnTc, where, (int)blockIdx.x);
+        return -1;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ int step_wait(uint32_t bar, uint32_t parity, volatile uint32_t* total,
+                                         uint32_t n, volatile int* abort_flag, WsHeader* hdr,
+                                         int where) {
+  if (mbar_try(bar, parity)) return 1;
+  return step_wait_slow(bar, parity, total, n, abort_flag, hdr, where);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
@@ -423,6 +456,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   volatile int* sAbort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   ItemSlot* sItem = reinterpret_cast<ItemSlot*>(smem + kOffMisc + 16);  // [stream][slot]
   volatile uint32_t* sStep = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc + 112);  // [stream][S buffer]
+  // step count of the whole walk, published by the K producer when it ends
+  volatile uint32_t* sTotal = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc + 8);
+  // per K stage and per P tile: stream and position of the step they hold
+  volatile uint32_t* sKMeta = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc + 128);  // [2]
+  volatile uint32_t* sPMeta = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc + 136);  // [kPTiles]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   auto bar = [&](int idx) { return bars + 8u * idx; };
@@ -431,7 +469,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int x = 0; x < kStreams; ++x) {
       for (int u = 0; u < 2; ++u) {
         mbar_init(bar(B_ITEM_FULL + 2 * x + u), 1);
-        mbar_init(bar(B_ITEM_EMPTY + 2 * x + u), 4);
+        mbar_init(bar(B_ITEM_EMPTY + 2 * x + u), 2);  // V producer + softmax
         mbar_init(bar(B_S_FULL + 2 * x + u), 2);  // MMA commit + step-id publication
         mbar_init(bar(B_S_FREE + 2 * x + u), 128);
       }
@@ -448,6 +486,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(bar(B_P_EMPTY + t), 1);
     }
     *sAbort = 0;
+    *sTotal = 0xffffffffu;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -562,6 +601,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const uint32_t prev = (kuse >> (8 * ks)) & 0xffu;
           if (prev & 1u) ok = ok && mbar_wait(bar(B_S_FULL + (prev >> 2)), (prev >> 1) & 1u, sAbort, a.hdr, 3);
           if (ok) {
+            sKMeta[ks] = step_meta(x, c == 0, c == wk.C.get(x) - 1, nblk);
             mbar_expect_tx(bar(B_K_FULL + ks), nblk * (kKVBytes / 2));
             const uint32_t dk = sbase + kOffK + ks * kKVBytes;
             for (int bb = 0; bb < nblk; ++bb) {
@@ -581,6 +621,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
         wk.advance(x);
       }
+      if (lane == 0) *sTotal = gk;
       // drain: every issued load has landed before the CTA may exit
       if (lane == 0) {
         volatile int no_abort = 0;
@@ -650,42 +691,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // ---------------------------------------------------------------- MMA issuers
       const bool is_s = warp == 1;
       if (lane == 0) {
-        uint32_t gk = 0, gv = 0;
         Pair<uint32_t> gs = {0u, 0u};   // S^T uses per stream (buffer = gs & 1)
         Pair<uint32_t> gq = {0u, 0u};   // Q tiles per stream
-        Pair<uint32_t> gp = {0u, 0u};   // P tiles per stream
-        Pair<int> nkept = {0, 0};
         bool ok = true;
-        Walk wk;
-        wk.init();
         // descriptor templates: k-steps only advance the 14-bit start-address field
         const uint64_t dK0 = smem_desc(sbase + kOffK, 16, 1024);
         const uint64_t dQ0 = smem_desc(sbase + kOffQ, 16, 1024);
         const uint64_t dV0 = smem_desc(sbase + kOffV, kKVBytes / 2, 1024);
         const uint64_t dP0 = smem_desc(sbase + kOffP, kPBytes, 1024);
-        for (;;) {
-          const int x = wk.pick();
-          if (x < 0) break;
-          if (wk.C.get(x) < 0) {
-            const int tx = wk.t.get(x);
-            const int slot = tx & 1;
-            ok = ok && mbar_wait(bar(B_ITEM_FULL + 2 * x + slot), (tx >> 1) & 1, sAbort, a.hdr, 12);
-            const int n = ok ? sItem[2 * x + slot].n : -1;
-            mbar_arrive(bar(B_ITEM_EMPTY + 2 * x + slot));
-            if (n < 0) {
-              wk.done.set(x, 1);
-              continue;
-            }
-            nkept.set(x, n);
-            wk.open(x, n);
-            if (n > 0 && is_s) ok = ok && mbar_wait(bar(B_Q_FULL + x), gq.inc(x) & 1, sAbort, a.hdr, 13);
-            continue;
-          }
-          const int c = wk.c.get(x);
+        // Walk step n: its stream and item position come with its data, from the
+        // K producer beside the K stage (S^T issuer) and from the softmax beside
+        // the P tile (PV issuer).
+        uint32_t n = 0;
+        for (;; ++n) {
           if (is_s) {
+            const uint32_t ks = n & 1;
+            const int w = step_wait(bar(B_K_FULL + ks), (n >> 1) & 1, sTotal, n, sAbort, a.hdr, 14);
+            if (w <= 0) break;
+            const uint32_t meta = sKMeta[ks];
+            const int x = (int)(meta & 1u);
             const uint32_t gsx = gs.get(x);
-            const uint32_t ks = gk & 1, sb = gsx & 1;
-            ok = ok && mbar_wait(bar(B_K_FULL + ks), (gk >> 1) & 1, sAbort, a.hdr, 14);
+            const uint32_t sb = gsx & 1;
+            if (meta & 2u) ok = ok && mbar_wait(bar(B_Q_FULL + x), gq.inc(x) & 1, sAbort, a.hdr, 13);
             if (gsx >= 2)
               ok = ok && mbar_wait(bar(B_S_FREE + 2 * x + sb), ((gsx >> 1) - 1) & 1, sAbort, a.hdr, 15);
             tc_fence_after();
@@ -699,35 +726,36 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                        dq + (uint64_t)(((kk >> 2) * (kQBytes / 2) + (kk & 3) * 32) >> 4), kIdescS,
                        kk > 0 ? 1u : 0u);
             }
-            sStep[2 * x + sb] = gk;
+            sStep[2 * x + sb] = n;
             tc_commit(bar(B_S_FULL + 2 * x + sb));  // also frees K stage ks
             mbar_arrive(bar(B_S_FULL + 2 * x + sb));  // releases the step id
-            if (c == wk.C.get(x) - 1) tc_commit(bar(B_Q_EMPTY + x));
-            ++gk;
+            if (meta & 4u) tc_commit(bar(B_Q_EMPTY + x));
             gs.inc(x);
           } else {
-            const uint32_t vs = gv & 1;
-            const uint32_t pt = gv % kPTiles, pu = gv / kPTiles;
-            ok = ok && mbar_wait(bar(B_P_FULL + pt), pu & 1, sAbort, a.hdr, 10);
-            ok = ok && mbar_wait(bar(B_V_FULL + vs), (gv >> 1) & 1, sAbort, a.hdr, 11);
+            const uint32_t vs = n & 1;
+            const uint32_t pt = n % kPTiles, pu = n / kPTiles;
+            const int w = step_wait(bar(B_P_FULL + pt), pu & 1, sTotal, n, sAbort, a.hdr, 10);
+            if (w <= 0) break;
+            const uint32_t meta = sPMeta[pt];
+            const int x = (int)(meta & 1u);
+            ok = ok && mbar_wait(bar(B_V_FULL + vs), (n >> 1) & 1, sAbort, a.hdr, 11);
             tc_fence_after();
             if (ok) {
-              const int ksteps = min(2, nkept.get(x) - 2 * c) * (kBS / 16);
+              const int ksteps = (int)(meta >> 3) * (kBS / 16);
+              const uint32_t acc0 = (meta & 2u) ? 0u : 1u;
               const uint64_t dv = dV0 + (uint64_t)((vs * kKVBytes) >> 4);
               const uint64_t dp = dP0 + (uint64_t)((pt * kPBytes) >> 4);
               const uint32_t d = tmem + col_o(x);
               for (int kk = 0; kk < ksteps; ++kk)
                 tc_mma(d, dv + (uint64_t)(kk * 128), dp + (uint64_t)(kk * 128), kIdescPV,
-                       (c > 0 || kk > 0) ? 1u : 0u);
+                       kk > 0 ? 1u : acc0);
             }
             tc_commit(bar(B_P_EMPTY + pt));
             tc_commit(bar(B_V_EMPTY + vs));
-            if (c == wk.C.get(x) - 1) tc_commit(bar(B_O_DONE + x));
-            ++gv;
-            gp.inc(x);
+            if (meta & 4u) tc_commit(bar(B_O_DONE + x));
           }
-          wk.advance(x);
         }
+        const uint32_t gv = n;
         // the tensor core has finished every MMA before TMEM is released
         volatile int no_abort = 0;
         if (!is_s && gv > 0)
@@ -904,6 +932,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
+        if (r == 0) sPMeta[n_step % kPTiles] = step_meta(x, c == 0, c == C - 1, nblk);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
         mbar_arrive(bar(B_P_FULL + n_step % kPTiles));
