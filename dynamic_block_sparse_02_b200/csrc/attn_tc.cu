@@ -90,9 +90,9 @@ enum {
   B_Q_FULL = 8,       // [2]
   B_Q_EMPTY = 10,     // [2]
   B_K_FULL = 12,      // [2]
-  B_K_EMPTY = 14,     // [2]
+  B_K_EMPTY = 14,     // [2] spare: a K stage is free once its S^T has completed (S_FULL)
   B_V_FULL = 16,      // [2]
-  B_V_EMPTY = 18,     // [2]
+  B_V_EMPTY = 18,     // [2] spare: a V stage is free once its PV has completed (P_EMPTY)
   B_S_FULL = 20,      // [2][2]
   B_S_FREE = 24,      // [2][2]
   B_P_FULL = 28,      // [kPTiles]
@@ -305,9 +305,16 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ void add_bf16_pair(float& lo, float& hi, uint32_t w) {
-  lo += __uint_as_float(w << 16);
-  hi += __uint_as_float(w & 0xffff0000u);
+// c + (low / high bf16 half of w), one mixed-precision add (fp32 result, round to nearest)
+__device__ __forceinline__ float add_lo(float c, uint32_t w) {
+  float d;
+  asm("{ .reg .b16 lo, hi; mov.b32 {lo, hi}, %1; add.rn.f32.bf16 %0, lo, %2; }" : "=f"(d) : "r"(w), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float add_hi(float c, uint32_t w) {
+  float d;
+  asm("{ .reg .b16 lo, hi; mov.b32 {lo, hi}, %1; add.rn.f32.bf16 %0, hi, %2; }" : "=f"(d) : "r"(w), "f"(c));
+  return d;
 }
 
 // Named barrier over the 128 threads of one softmax warpgroup (id 1 + stream),
@@ -666,7 +673,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const int slot = wk.t.get(x) & 1;
           const int nblk = min(2, nkept.get(x) - 2 * c);
           const uint32_t vs = gv & 1;
-          if (gv >= 2) ok = ok && mbar_wait(bar(B_V_EMPTY + vs), ((gv >> 1) - 1) & 1, sAbort, a.hdr, 4);
+          // the stage's previous tile belongs to step gv - 2, whose PV also freed its P tile
+          if (gv >= 2)
+            ok = ok && mbar_wait(bar(B_P_EMPTY + (gv - 2) % kPTiles), ((gv - 2) / kPTiles) & 1, sAbort, a.hdr, 4);
           if (ok) {
             const int16_t* my_list = lists + (2 * x + slot) * kMaxBlocks;
             const int kvr = kvrow.get(x);
@@ -746,12 +755,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               const uint64_t dv = dV0 + (uint64_t)((vs * kKVBytes) >> 4);
               const uint64_t dp = dP0 + (uint64_t)((pt * kPBytes) >> 4);
               const uint32_t d = tmem + col_o(x);
-              for (int kk = 0; kk < ksteps; ++kk)
-                tc_mma(d, dv + (uint64_t)(kk * 128), dp + (uint64_t)(kk * 128), kIdescPV,
-                       kk > 0 ? 1u : acc0);
+              if (ksteps == 2 * (kBS / 16)) {
+#pragma unroll
+                for (int kk = 0; kk < 2 * (kBS / 16); ++kk)
+                  tc_mma(d, dv + (uint64_t)(kk * 128), dp + (uint64_t)(kk * 128), kIdescPV,
+                         kk > 0 ? 1u : acc0);
+              } else {
+#pragma unroll
+                for (int kk = 0; kk < kBS / 16; ++kk)
+                  tc_mma(d, dv + (uint64_t)(kk * 128), dp + (uint64_t)(kk * 128), kIdescPV,
+                         kk > 0 ? 1u : acc0);
+              }
             }
-            tc_commit(bar(B_P_EMPTY + pt));
-            tc_commit(bar(B_V_EMPTY + vs));
+            tc_commit(bar(B_P_EMPTY + pt));  // frees P tile pt and V stage vs
             if (meta & 4u) tc_commit(bar(B_O_DONE + x));
           }
         }
@@ -927,7 +943,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 p1 = kl > q + 1 ? 0.f : p1;
               }
               w[e] = pack_bf16(p0, p1);
-              l2[q >> 1] = __fadd2_rn(l2[q >> 1], make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u)));
+              l2[q >> 1].x = add_lo(l2[q >> 1].x, w[e]);
+              l2[q >> 1].y = add_hi(l2[q >> 1].y, w[e]);
             }
             *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
