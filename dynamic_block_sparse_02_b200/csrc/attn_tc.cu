@@ -926,12 +926,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
         } else {
           const float2 c22 = make_float2(c2, c2);
+          // The maxima of group cc + 1 are read before the P store of group cc:
+          // a shared load that follows a shared store would wait for it.
+          float4 n0 = reinterpret_cast<const float4*>(sNM)[0];
+          float4 n1 = reinterpret_cast<const float4*>(sNM)[1];
 #pragma unroll
           for (int cc = 0; cc < 8; ++cc) {
-            const float4 n0 = reinterpret_cast<const float4*>(sNM)[2 * cc];
-            const float4 n1 = reinterpret_cast<const float4*>(sNM)[2 * cc + 1];
             const float2 nm[4] = {make_float2(n0.x, n0.y), make_float2(n0.z, n0.w), make_float2(n1.x, n1.y),
                                   make_float2(n1.z, n1.w)};
+            if (cc < 7) {
+              n0 = reinterpret_cast<const float4*>(sNM)[2 * cc + 2];
+              n1 = reinterpret_cast<const float4*>(sNM)[2 * cc + 3];
+            }
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
