@@ -79,14 +79,13 @@ def kept_flops(cnt_sum: int, block: int, d: int) -> float:
 
 
 def select_bytes(w) -> float:
-    """Algorithmic HBM bytes of steps 1-3: Q and K read once, pooled blocks
-    written and read once, index rows and counts written."""
+    """Algorithmic HBM bytes of steps 1-3: Q and K read once, index rows and
+    counts written. Intermediates (pooled blocks, scores) are not counted."""
     q = w.B * w.Hq * w.N * w.d * 2
     k = w.B * w.Hkv * w.N * w.d * 2
-    pooled = (w.B * w.Hq + w.B * w.Hkv) * w.nb * w.d * 4
     width = min(w.nb, w.k_free + w.local_window + w.n_sink)
     sel = w.B * w.Hq * w.nb * (width + 1) * 4
-    return q + k + 2 * pooled + sel
+    return q + k + sel
 
 
 def load_peaks():

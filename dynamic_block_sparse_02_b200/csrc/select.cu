@@ -88,36 +88,6 @@ pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict
   }
 }
 
-// ---------------------------------------------------------------------------
-// Step 2: the block score of one pooled query row and one pooled key row.
-// Four fp32 partial sums over d (d = 4t+0 .. 4t+3), fused multiply-adds in
-// increasing t, combined as (x + y) + (z + w). Every kernel that produces a
-// score calls this function, so the split and the fused paths agree bit for
-// bit.
-// ---------------------------------------------------------------------------
-template <int D, int R>
-__device__ __forceinline__ void score_rows(const float* __restrict__ qs /*smem [R][D]*/,
-                                           const float* __restrict__ kp_row, float (&out)[R]) {
-  float4 a[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) a[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float4* k4 = reinterpret_cast<const float4*>(kp_row);
-#pragma unroll 4
-  for (int t = 0; t < D / 4; ++t) {
-    const float4 kv = __ldg(k4 + t);
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const float4 qv = reinterpret_cast<const float4*>(qs + r * D)[t];
-      a[r].x = __fmaf_rn(qv.x, kv.x, a[r].x);
-      a[r].y = __fmaf_rn(qv.y, kv.y, a[r].y);
-      a[r].z = __fmaf_rn(qv.z, kv.z, a[r].z);
-      a[r].w = __fmaf_rn(qv.w, kv.w, a[r].w);
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < R; ++r) out[r] = __fadd_rn(__fadd_rn(a[r].x, a[r].y), __fadd_rn(a[r].z, a[r].w));
-}
-
 // Map a score to an unsigned key whose order is the fp32 order (-0 == +0).
 // Every finite score maps to a key >= 0x00800000, so 0 can mark "not a
 // candidate".
@@ -129,25 +99,27 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
 
 // ---------------------------------------------------------------------------
 // Step 3: selection of one row (b, h, i) by one warp.
-// s: the row's scores s[0..i] (shared memory); skey: per-warp scratch of at
-// least i+1 words. Writes idx_row[0..W) (kept blocks ascending, then -1) and
-// *cnt_out.
+// s: the row's scores s[0..i] (shared memory); hist: 256 words of per-warp
+// scratch. Writes idx_row[0..W) (kept blocks ascending, then -1) and *cnt_out.
+// TMAX >= ceil((i+1)/32) bounds the blocks per lane.
 //
 // Candidates are the causal blocks outside the forced set; lane l owns blocks
-// l, l+32, l+64, ... The k best (larger fp32 score first, lower block index on
-// ties) are found in three steps:
+// l, l+32, l+64, ..., whose order-preserving keys it keeps in registers. The k
+// best (larger fp32 score first, lower block index on ties) are found as:
 //  1. a lower bound L on the k-th best key: with r = ceil(k/32), every lane's
 //     r-th largest key is >= the minimum of those over the warp, so at least
-//     32r >= k keys are >= L (L = 0, no bound, when some lane has fewer than
-//     r candidates or r > 4);
-//  2. the candidates with key >= L ("survivors") are compacted into skey;
-//  3. a most-significant-bit-first radix select over the survivors, starting
-//     at the highest bit in which they differ, finds the threshold prefix;
-//     equal keys left at the end are taken in increasing block index.
+//     32r >= k keys are >= L (no bound when r > 4); keys >= L survive;
+//  2. a most-significant-digit-first radix select over the survivors, from the
+//     highest bit in which L and the largest key differ (the survivors agree on
+//     every bit above it), 8 bits per pass: a histogram of the
+//     current digit among survivors that match the prefix found so far picks
+//     the digit holding the k-th best; it stops once every matching survivor
+//     is needed;
+//  3. survivors above the prefix are kept, and of those matching it the
+//     lowest block indices, as many as still needed.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ bool is_forced(int j, int win_lo, int ns) { return j >= win_lo || j < ns; }
-
-__device__ void select_row(const float* s, uint32_t* skey, int i, int k, int lw, int ns, int W,
+template <int TMAX>
+__device__ void select_row(const float* s, uint32_t* hist, int i, int k, int lw, int ns, int W,
                            int32_t* __restrict__ idx_row, int32_t* __restrict__ cnt_out,
                            WsHeader* hdr, int lane) {
   const int n = i + 1;
@@ -158,90 +130,132 @@ __device__ void select_row(const float* s, uint32_t* skey, int i, int k, int lw,
   const int T = (n + 31) >> 5;
   const uint32_t lt = (1u << lane) - 1u;
 
-  uint32_t surv = 0;          // bit t: block lane + 32t is a survivor
-  uint32_t prefix = 0, pmask = 0;
-  int need = keff;
-  if (keff > 0 && keff < ncand) {
-    // 1. lower bound from each lane's r-th largest key
-    const int r = (keff + 31) >> 5;
-    uint32_t L = 0;
-    if (r <= 4) {
-      uint32_t t0 = 0, t1 = 0, t2 = 0, t3 = 0;  // this lane's largest keys, descending
-      for (int t = 0; t < T; ++t) {
-        const int j = t * 32 + lane;
-        if (j < n && !is_forced(j, win_lo, ns)) {
-          uint32_t v = ordered_key(s[j]), u;
-          u = max(t0, v); v = min(t0, v); t0 = u;
-          u = max(t1, v); v = min(t1, v); t1 = u;
-          u = max(t2, v); v = min(t2, v); t2 = u;
-          t3 = max(t3, v);
-        }
-      }
-      const uint32_t mine = r == 1 ? t0 : r == 2 ? t1 : r == 3 ? t2 : t3;
-      L = __reduce_min_sync(kFull, mine);
-    }
-    // 2. compact the survivors' keys
-    int m = 0;
-    for (int t = 0; t < T; ++t) {
-      const int j = t * 32 + lane;
-      uint32_t key = 0;
-      if (j < n && !is_forced(j, win_lo, ns)) key = ordered_key(s[j]);
-      const bool sv = key != 0u && key >= L;
-      const uint32_t bm = __ballot_sync(kFull, sv);
-      if (sv) skey[m + __popc(bm & lt)] = key;
-      surv |= (uint32_t)sv << t;
-      m += __popc(bm);
-    }
-    __syncwarp();
-    // 3. radix select over the survivors from their highest differing bit
-    const uint32_t k0 = skey[0];
-    uint32_t diff = 0;
-    for (int u = lane; u < m; u += 32) diff |= skey[u] ^ k0;
-    diff = __reduce_or_sync(kFull, diff);
-    if (diff == 0u) {
-      pmask = 0xffffffffu;  // all survivors equal: lowest indices win
-      prefix = k0;
-    } else {
-      const int hb = 31 - __clz(diff);
-      pmask = hb == 31 ? 0u : ~((2u << hb) - 1u);
-      prefix = k0 & pmask;
-      int msurv = m;
-      for (int bit = hb; bit >= 0 && msurv != need; --bit) {
-        const uint32_t bb = 1u << bit;
-        int c = 0;
-        for (int u = lane; u < m; u += 32) {
-          const uint32_t key = skey[u];
-          c += ((key & pmask) == prefix) & ((key & bb) != 0u);
-        }
-        c = __reduce_add_sync(kFull, c);
-        if (c >= need) {
-          prefix |= bb;
-          msurv = c;
-        } else {
-          need -= c;
-          msurv -= c;
-        }
-        pmask |= bb;
-      }
-    }
-  } else if (keff > 0) {
-    // every candidate is kept
-    for (int t = 0; t < T; ++t) {
-      const int j = t * 32 + lane;
-      surv |= (uint32_t)(j < n && !is_forced(j, win_lo, ns)) << t;
-    }
-    need = ncand;  // pmask = prefix = 0: every survivor matches
+  // candidates are ns <= j < win_lo (the forced blocks are j < ns and j >= win_lo)
+  uint32_t key[TMAX];  // 0: not a candidate (every finite score has a key >= 0x00800000)
+#pragma unroll
+  for (int t = 0; t < TMAX; ++t) {
+    key[t] = 0u;
+    if (t >= T) break;
+    const int j = t * 32 + lane;
+    if (j >= ns && j < win_lo) key[t] = ordered_key(s[j]);
   }
 
-  // emit forced blocks and picks in ascending block order
+  uint32_t L = 1u;               // survivors: key >= L
+  uint32_t prefix = 0, pmask = 0;
+  int need = keff;               // still to take among survivors matching the prefix
+  if (keff == 0) {
+    L = 0xffffffffu;             // nothing survives (0xffffffff is not a finite key)
+    need = 0;
+  } else if (keff < ncand) {
+    // 1. lower bound from each lane's r-th largest key; the largest key overall
+    const int r = (keff + 31) >> 5;
+    uint32_t kmax;
+    if (r <= 2) {
+      uint32_t t0 = 0, t1 = 0;  // this lane's two largest keys, descending
+#pragma unroll
+      for (int t = 0; t < TMAX; ++t) {
+        if (t >= T) break;
+        const uint32_t v = key[t];
+        t1 = max(t1, min(t0, v));
+        t0 = max(t0, v);
+      }
+      L = max(__reduce_min_sync(kFull, r == 1 ? t0 : t1), 1u);
+      kmax = __reduce_max_sync(kFull, t0);
+    } else if (r <= 4) {
+      uint32_t t0 = 0, t1 = 0, t2 = 0, t3 = 0;  // this lane's largest keys, descending
+#pragma unroll
+      for (int t = 0; t < TMAX; ++t) {
+        if (t >= T) break;
+        uint32_t v = key[t], u;
+        u = max(t0, v); v = min(t0, v); t0 = u;
+        u = max(t1, v); v = min(t1, v); t1 = u;
+        u = max(t2, v); v = min(t2, v); t2 = u;
+        t3 = max(t3, v);
+      }
+      L = max(__reduce_min_sync(kFull, r == 3 ? t2 : t3), 1u);
+      kmax = __reduce_max_sync(kFull, t0);
+    } else {
+      uint32_t m = 0;
+#pragma unroll
+      for (int t = 0; t < TMAX; ++t) {
+        if (t >= T) break;
+        m = max(m, key[t]);
+      }
+      kmax = __reduce_max_sync(kFull, m);
+    }
+    // 2. radix select; every survivor lies in [L, kmax], so the survivors agree
+    // on all bits above the highest bit in which L and kmax differ
+    const uint32_t diff = kmax ^ L;
+    if (diff == 0u) {
+      pmask = 0xffffffffu;  // all survivors equal: lowest indices win
+      prefix = kmax;
+    } else {
+      int top = 31 - __clz(diff);
+      pmask = top == 31 ? 0u : ~((2u << top) - 1u);
+      prefix = kmax & pmask;
+      while (top >= 0) {
+        const int lo = max(top - 7, 0);
+        const uint32_t dmask = (2u << (top - lo)) - 1u;
+        reinterpret_cast<uint4*>(hist)[2 * lane] = make_uint4(0u, 0u, 0u, 0u);
+        reinterpret_cast<uint4*>(hist)[2 * lane + 1] = make_uint4(0u, 0u, 0u, 0u);
+        __syncwarp();
+#pragma unroll
+        for (int t = 0; t < TMAX; ++t) {
+          if (t >= T) break;
+          if (key[t] >= L && (key[t] & pmask) == prefix) atomicAdd(&hist[(key[t] >> lo) & dmask], 1u);
+        }
+        __syncwarp();
+        // bins 8*lane .. 8*lane+7; counts above a bin come from higher lanes
+        const uint4 h0 = reinterpret_cast<const uint4*>(hist)[2 * lane];
+        const uint4 h1 = reinterpret_cast<const uint4*>(hist)[2 * lane + 1];
+        const uint32_t c[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+        const int tl = (int)(((c[0] + c[1]) + (c[2] + c[3])) + ((c[4] + c[5]) + (c[6] + c[7])));
+        int incl = tl;  // sum over lanes >= this one
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int y = __shfl_down_sync(kFull, incl, off);
+          if (lane + off < 32) incl += y;
+        }
+        const int excl = incl - tl;
+        const uint32_t owner = __ballot_sync(kFull, excl < need && need <= incl);
+        const int ol = owner ? __ffs(owner) - 1 : 0;
+        int dg = 0, above = excl, cnt_dg = 0;
+        if (lane == ol) {
+#pragma unroll
+          for (int b = 7; b >= 0; --b) {
+            if (above + (int)c[b] >= need) {
+              dg = 8 * lane + b;
+              cnt_dg = (int)c[b];
+              break;
+            }
+            above += (int)c[b];
+          }
+        }
+        dg = __shfl_sync(kFull, dg, ol);
+        above = __shfl_sync(kFull, above, ol);
+        cnt_dg = __shfl_sync(kFull, cnt_dg, ol);
+        need -= above;
+        prefix |= (uint32_t)dg << lo;
+        pmask |= dmask << lo;
+        if (cnt_dg == need) break;  // every survivor matching the prefix is taken
+        top = lo - 1;
+        __syncwarp();
+      }
+    }
+  } else {
+    need = ncand;  // every candidate is kept: L = 1, pmask = prefix = 0
+  }
+
+  // 3. emit forced blocks and picks in ascending block order
   int base = 0, rank_base = 0;
-  for (int t = 0; t < T; ++t) {
+#pragma unroll
+  for (int t = 0; t < TMAX; ++t) {
+    if (t >= T) break;
     const int j = t * 32 + lane;
-    const bool forced = j < n && is_forced(j, win_lo, ns);
-    const bool sv = (surv >> t) & 1u;
-    const uint32_t key = sv ? ordered_key(s[j]) : 0u;
-    const bool above = sv && ((key & pmask) > prefix);
-    const bool match = sv && ((key & pmask) == prefix);
+    const bool forced = j < n && (j < ns || j >= win_lo);
+    const bool sv = key[t] >= L;  // L >= 1, so non-candidates (key 0) never survive
+    const bool above = sv && ((key[t] & pmask) > prefix);
+    const bool match = sv && ((key[t] & pmask) == prefix);
     const uint32_t mm = __ballot_sync(kFull, match);
     const int rk = rank_base + __popc(mm & lt);
     rank_base += __popc(mm);
@@ -259,8 +273,24 @@ __device__ void select_row(const float* s, uint32_t* skey, int i, int k, int lw,
   __syncwarp();
 }
 
-// Rows handled by one CTA of the score kernels: heads [h0, h0+HB) of one KV
-// group (all share pooled K) times query blocks [i0, i0+RB), HB*RB <= 8.
+// ---------------------------------------------------------------------------
+// Step 2 (+3 when FUSED): one CTA scores kRowTile pooled query rows against the
+// pooled key rows 0..jmax of their KV head, as a tiled fp32 GEMM, then selects
+// each row from the scores held in shared memory (or writes them out).
+// Rows are heads [h0, h0+HB) of one KV group times query blocks [i0, i0+RB),
+// HB * RB <= kRowTile. A score is the fp32 sum of two fused multiply-add
+// chains, over the even and over the odd d in increasing order; both the fused
+// and the split path run this kernel, so they agree bit for bit.
+// ---------------------------------------------------------------------------
+constexpr int kRowTile = 32;   // query rows per CTA
+constexpr int kColTile = 128;  // key blocks per column pass
+constexpr int kDTile = 32;     // head-dim slice per pass over the key tile
+template <int D>
+struct QStride {
+  static constexpr int value = D + 4;
+};
+constexpr int kKStride = kDTile + 4;
+
 struct RowTile {
   int b, kvh, h0, i0;
 };
@@ -284,61 +314,137 @@ __device__ __forceinline__ RowTile row_tile(const Shape& s, int HB, int RB) {
   return t;
 }
 
-// Scores of the CTA's rows against key blocks 0..jmax into shared memory;
-// then either the fused selection (FUSED) or a plain copy to `scores`.
-template <int D, bool FUSED>
+constexpr int kHistWords = 256;  // per-warp radix histogram of the selection
+
+// Shared memory: qs [kRowTile][D+4] and ks [kColTile][kDTile+4] during the
+// GEMM, reused as the selection histograms [kSelWarps][256] afterwards; then
+// sc [kRowTile][nb].
+template <int D>
+size_t score_smem_bytes(int nb) {
+  const size_t gemm = (size_t)(kRowTile * QStride<D>::value + kColTile * kKStride) * sizeof(float);
+  static_assert((size_t)(kRowTile * QStride<D>::value + kColTile * kKStride) >= (size_t)kSelWarps * kHistWords,
+                "the histograms fit in the GEMM buffers");
+  return gemm + (size_t)kRowTile * nb * sizeof(float);
+}
+
+// Blocks per lane of a selection row: ceil(nb / 32) rounded up to 8, 16 or 32.
+inline int select_tmax(int nb) { return nb <= 256 ? 8 : nb <= 512 ? 16 : 32; }
+
+template <int D, bool FUSED, int TMAX>
 __global__ void __launch_bounds__(kSelThreads)
 score_kernel(Shape s, KBudget kb, int HB, int RB, const float* __restrict__ qp,
              const float* __restrict__ kp, float* __restrict__ scores, int32_t* __restrict__ idx,
              int32_t* __restrict__ cnt, WsHeader* hdr) {
   extern __shared__ float sm_f[];
-  float* qs = sm_f;                       // [8][D]
-  float* sc = sm_f + kSelWarps * D;       // [8][nb]
-  uint32_t* sk = reinterpret_cast<uint32_t*>(sc + kSelWarps * s.nb);  // [8][nb] (FUSED only)
+  constexpr int QS = QStride<D>::value;
+  float* const qs = sm_f;                                   // [kRowTile][QS]
+  float* const ks = sm_f + kRowTile * QS;                   // [kColTile][kKStride]
+  const size_t lead = (size_t)kRowTile * QS + kColTile * kKStride;
+  uint32_t* const sk = reinterpret_cast<uint32_t*>(sm_f);  // [kSelWarps][256], after the GEMM
+  float* const sc = sm_f + lead;                            // [kRowTile][nb]
   const RowTile tile = row_tile(s, HB, RB);
   const int h_end = min(tile.h0 + HB, (tile.kvh + 1) * s.group);
   const int i_end = min(tile.i0 + RB, s.nb);
+  const int tid = threadIdx.x;
 
-  // slot r -> (h, i); inactive slots hold zeros and are never read back
-  for (int e = threadIdx.x; e < kSelWarps * D; e += kSelThreads) {
-    const int r = e / D, c = e % D;
+  // tile row r -> (h, i); rows outside the problem hold zeros and are never read back
+  for (int e = tid; e < kRowTile * (D / 4); e += kSelThreads) {
+    const int r = e / (D / 4), c4 = e % (D / 4);
     const int h = tile.h0 + r / RB, i = tile.i0 + r % RB;
-    float v = 0.f;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r < HB * RB && h < h_end && i < i_end)
-      v = qp[(((size_t)tile.b * s.Hq + h) * s.nb + i) * D + c];
-    qs[e] = v;
+      v = *reinterpret_cast<const float4*>(qp + (((size_t)tile.b * s.Hq + h) * s.nb + i) * D + 4 * c4);
+    *reinterpret_cast<float4*>(qs + r * QS + 4 * c4) = v;
   }
-  __syncthreads();
 
+  // thread (rg, cg) owns rows rg + 8u (u < 4) and columns cg + 32v (v < 4) of
+  // each column pass; the strides keep the shared loads free of bank conflicts
+  const int rg = tid % 8, cg = tid / 8;
   const int jmax = i_end - 1;
-  const float* kbase = kp + ((size_t)tile.b * s.Hkv + tile.kvh) * s.nb * D;
-  for (int j = threadIdx.x; j <= jmax; j += kSelThreads) {
-    float o[kSelWarps];
-    score_rows<D, kSelWarps>(qs, kbase + (size_t)j * D, o);
+  const float* const kbase = kp + ((size_t)tile.b * s.Hkv + tile.kvh) * s.nb * D;
+  // the key tile streams through shared memory one (column pass, d slice) at a
+  // time; the next slice is fetched into registers while this one is used
+  constexpr int kSlices = D / kDTile;
+  constexpr int kLoads = kColTile * (kDTile / 4) / kSelThreads;  // float4 per thread per slice
+  const int n_pass = jmax / kColTile + 1;
+  float4 nxt[kLoads];
+  auto fetch = [&](int pass, int slice) {
 #pragma unroll
-    for (int r = 0; r < kSelWarps; ++r) {
+    for (int u = 0; u < kLoads; ++u) {
+      const int e = tid + u * kSelThreads;
+      const int col = e / (kDTile / 4), d4 = e % (kDTile / 4);
+      const int j = pass * kColTile + col;
+      nxt[u] = j <= jmax ? __ldg(reinterpret_cast<const float4*>(kbase + (size_t)j * D + slice * kDTile) + d4)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  fetch(0, 0);
+  for (int pass = 0; pass < n_pass; ++pass) {
+    const int jc = pass * kColTile;
+    float2 acc[4][4];  // partial sums over even and odd d
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[u][v] = make_float2(0.f, 0.f);
+    for (int sl = 0; sl < kSlices; ++sl) {
+      __syncthreads();  // the previous slice has been consumed (and qs is complete)
+#pragma unroll
+      for (int u = 0; u < kLoads; ++u) {
+        const int e = tid + u * kSelThreads;
+        const int col = e / (kDTile / 4), d4 = e % (kDTile / 4);
+        *reinterpret_cast<float4*>(ks + col * kKStride + 4 * d4) = nxt[u];
+      }
+      __syncthreads();
+      if (sl + 1 < kSlices) fetch(pass, sl + 1);
+      else if (pass + 1 < n_pass) fetch(pass + 1, 0);
+      const int dc = sl * kDTile;
+#pragma unroll 2
+      for (int d4 = 0; d4 < kDTile / 4; ++d4) {
+        float4 qv[4], kv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) qv[u] = *reinterpret_cast<const float4*>(qs + (rg + 8 * u) * QS + dc + 4 * d4);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) kv[v] = *reinterpret_cast<const float4*>(ks + (cg + 32 * v) * kKStride + 4 * d4);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            acc[u][v] = __ffma2_rn(make_float2(qv[u].x, qv[u].y), make_float2(kv[v].x, kv[v].y), acc[u][v]);
+            acc[u][v] = __ffma2_rn(make_float2(qv[u].z, qv[u].w), make_float2(kv[v].z, kv[v].w), acc[u][v]);
+          }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = rg + 8 * u;
       const int i = tile.i0 + r % RB;
-      sc[r * s.nb + j] = (j <= i) ? o[r] : -INFINITY;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int j = jc + cg + 32 * v;
+        if (j <= jmax) sc[r * s.nb + j] = (j <= i) ? __fadd_rn(acc[u][v].x, acc[u][v].y) : -INFINITY;
+      }
     }
   }
-  __syncthreads();
+  __syncthreads();  // all scores written; qs/ks are free for the selection scratch
 
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int r = warp;
-  const int h = tile.h0 + r / RB, i = tile.i0 + r % RB;
-  if (r >= HB * RB || h >= h_end || i >= i_end) return;
-  const size_t row = ((size_t)tile.b * s.Hq + h) * s.nb + i;
-  if (FUSED) {
-    const int k = s.per_head ? kb.k[h] : kb.k[0];
-    select_row(sc + r * s.nb, sk + r * s.nb, i, k, s.lw, s.ns, s.W, idx + row * s.W, cnt + row, hdr,
-               lane);
-  } else {
-    float* dst = scores + row * s.nb;
-    for (int j = lane; j < s.nb; j += 32) dst[j] = (j <= i) ? sc[r * s.nb + j] : -INFINITY;
+  const int warp = tid / 32, lane = tid % 32;
+  for (int r = warp; r < kRowTile; r += kSelWarps) {
+    const int h = tile.h0 + r / RB, i = tile.i0 + r % RB;
+    if (r >= HB * RB || h >= h_end || i >= i_end) continue;
+    const size_t row = ((size_t)tile.b * s.Hq + h) * s.nb + i;
+    if (FUSED) {
+      const int k = s.per_head ? kb.k[h] : kb.k[0];
+      select_row<TMAX>(sc + r * s.nb, sk + warp * kHistWords, i, k, s.lw, s.ns, s.W, idx + row * s.W,
+                       cnt + row, hdr, lane);
+    } else {
+      float* dst = scores + row * s.nb;
+      for (int j = lane; j < s.nb; j += 32) dst[j] = (j <= i) ? sc[r * s.nb + j] : -INFINITY;
+    }
   }
 }
 
 // Selection on caller scores: one warp per row (b, h, i).
+template <int TMAX>
 __global__ void __launch_bounds__(kSelThreads)
 select_kernel(Shape s, KBudget kb, const float* __restrict__ scores, int32_t* __restrict__ idx,
               int32_t* __restrict__ cnt, WsHeader* hdr, long long n_rows) {
@@ -349,17 +455,17 @@ select_kernel(Shape s, KBudget kb, const float* __restrict__ scores, int32_t* __
   const int i = (int)(row % s.nb);
   const int h = (int)((row / s.nb) % s.Hq);
   float* sc = sm_f + warp * s.nb;
-  uint32_t* sk = reinterpret_cast<uint32_t*>(sm_f + kSelWarps * s.nb) + warp * s.nb;
+  uint32_t* sk = reinterpret_cast<uint32_t*>(sm_f + kSelWarps * s.nb) + warp * kHistWords;
   const float* src = scores + (size_t)row * s.nb;
   for (int j = lane; j <= i; j += 32) sc[j] = src[j];
   __syncwarp();
   const int k = s.per_head ? kb.k[h] : kb.k[0];
-  select_row(sc, sk, i, k, s.lw, s.ns, s.W, idx + (size_t)row * s.W, cnt + row, hdr, lane);
+  select_row<TMAX>(sc, sk, i, k, s.lw, s.ns, s.W, idx + (size_t)row * s.W, cnt + row, hdr, lane);
 }
 
 void row_tiling(const Shape& s, int& HB, int& RB) {
-  HB = s.group < kSelWarps ? s.group : kSelWarps;
-  RB = kSelWarps / HB;
+  HB = s.group < kRowTile ? s.group : kRowTile;
+  RB = kRowTile / HB;
   if (RB < 1) RB = 1;
 }
 
@@ -369,26 +475,27 @@ int score_grid(const Shape& s, int HB, int RB) {
   return s.B * s.Hkv * n_hc * n_ic;
 }
 
+template <int D, bool FUSED>
+cudaError_t launch_score_d(const Shape& s, const KBudget& kb, const float* qp, const float* kp,
+                           float* scores, int32_t* idx, int32_t* cnt, WsHeader* hdr, cudaStream_t st) {
+  int HB, RB;
+  row_tiling(s, HB, RB);
+  const size_t smem = score_smem_bytes<D>(s.nb);
+  const int grid = score_grid(s, HB, RB);
+  auto f = select_tmax(s.nb) == 8 ? score_kernel<D, FUSED, 8>
+           : select_tmax(s.nb) == 16 ? score_kernel<D, FUSED, 16> : score_kernel<D, FUSED, 32>;
+  cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  f<<<grid, kSelThreads, smem, st>>>(s, kb, HB, RB, qp, kp, scores, idx, cnt, hdr);
+  return cudaGetLastError();
+}
+
 template <bool FUSED>
 cudaError_t launch_score_impl(const Shape& s, const KBudget& kb, const float* qp, const float* kp,
                               float* scores, int32_t* idx, int32_t* cnt, WsHeader* hdr,
                               cudaStream_t st) {
-  int HB, RB;
-  row_tiling(s, HB, RB);
-  const size_t smem = (size_t)kSelWarps * (s.d + (FUSED ? 2 : 1) * s.nb) * sizeof(float);
-  const int grid = score_grid(s, HB, RB);
-  if (s.d == 64) {
-    auto f = score_kernel<64, FUSED>;
-    cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    f<<<grid, kSelThreads, smem, st>>>(s, kb, HB, RB, qp, kp, scores, idx, cnt, hdr);
-  } else {
-    auto f = score_kernel<128, FUSED>;
-    cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    f<<<grid, kSelThreads, smem, st>>>(s, kb, HB, RB, qp, kp, scores, idx, cnt, hdr);
-  }
-  return cudaGetLastError();
+  if (s.d == 64) return launch_score_d<64, FUSED>(s, kb, qp, kp, scores, idx, cnt, hdr, st);
+  return launch_score_d<128, FUSED>(s, kb, qp, kp, scores, idx, cnt, hdr, st);
 }
 
 }  // namespace
@@ -429,11 +536,11 @@ cudaError_t launch_select(const Shape& s, const KBudget& kb, const float* scores
                           int32_t* cnt, WsHeader* hdr, cudaStream_t st) {
   const long long n_rows = (long long)s.B * s.Hq * s.nb;
   const long long grid = (n_rows + kSelWarps - 1) / kSelWarps;
-  const size_t smem = (size_t)kSelWarps * 2 * s.nb * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  const size_t smem = (size_t)kSelWarps * (s.nb + kHistWords) * sizeof(float);
+  auto f = select_tmax(s.nb) == 8 ? select_kernel<8> : select_tmax(s.nb) == 16 ? select_kernel<16> : select_kernel<32>;
+  cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  select_kernel<<<(unsigned)grid, kSelThreads, smem, st>>>(s, kb, scores, idx, cnt, hdr, n_rows);
+  f<<<(unsigned)grid, kSelThreads, smem, st>>>(s, kb, scores, idx, cnt, hdr, n_rows);
   return cudaGetLastError();
 }
 
