@@ -21,6 +21,9 @@ What is computed, and where the pages say so:
   ranking is taken on fp32 scores, because the "DeepSeek NSA" article, section
   2.2, keeps the routing decision in FP32; the oracle rounds its fp64 score to
   fp32 once and ranks on that, ties going to the lower block index.
+* Group-shared selection (an alternative rule): one list per KV head, chosen
+  by the same rule from the sum of its query heads' block scores and used by
+  all of them (see group_scores).
 * Attention. softmax(Q K^T * scale) V over the kept key blocks only, with the
   causal mask inside the diagonal block ("稀疏注意力 vs Flash Attention v2",
   section 1 pseudocode: scores, then the sparsity pattern, then softmax with
@@ -161,6 +164,44 @@ def select_blocks(scores: np.ndarray, k_free, local_window: int, n_sink: int,
                     raise ValueError("row width too small for the kept set")
                 idx[b, h, i, :len(kept)] = kept
                 cnt[b, h, i] = len(kept)
+    return idx, cnt
+
+
+def group_scores(scores: np.ndarray, group: int) -> np.ndarray:
+    """Scores of the group-shared rule: for KV head g, the sum over its query
+    heads h = g*group .. g*group+group-1 of their block scores (fp64, -inf
+    above the diagonal). Returns [B, Hq/group, nb, nb].
+
+    Follows the zblog.xzdbk.com/559 post (section on speculative decoding:
+    with MQA/GQA the shared KV cache lowers the cost of keeping the sparse
+    index) and the DSA post, section 2.1 (the indexer merges the lists of its
+    index heads). The pages give no rule for combining the heads; the plain
+    reading used here is the sum of the heads' block scores.
+    """
+    B, Hq, nb, _ = scores.shape
+    if Hq % group:
+        raise ValueError("Hq must be a multiple of the group size")
+    s = scores.reshape(B, Hq // group, group, nb, nb)
+    out = np.zeros((B, Hq // group, nb, nb), dtype=np.float64)
+    for u in range(group):
+        out += s[:, :, u]
+    return out
+
+
+def select_blocks_group(scores: np.ndarray, group: int, k_free: int, local_window: int,
+                        n_sink: int, width: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Group-shared selection: one kept list per (b, KV head, query block),
+    chosen by the same rule as select_blocks from the group's summed scores,
+    and given to every query head of the group.
+
+    Returns idx int32 [B,Hq,nb,width] and cnt int32 [B,Hq,nb] like
+    select_blocks, with identical rows for the heads of a group.
+    """
+    B, Hq, nb, _ = scores.shape
+    gs = group_scores(scores, group)
+    idx_g, cnt_g = select_blocks(gs, int(k_free), local_window, n_sink, width)
+    idx = np.repeat(idx_g, group, axis=1)
+    cnt = np.repeat(cnt_g, group, axis=1)
     return idx, cnt
 
 

@@ -368,3 +368,67 @@ def test_attended_pairs_dense_causal():
     for i in range(nb):
         idx[0, 0, i, i + 1:] = -1
     assert oracle.attended_pairs(idx, cnt, bs) == oracle.dense_pairs(N, causal=True)
+
+
+# ---------------------------------------------------------------------------
+# Group-shared selection (one list per KV head from the summed head scores)
+# ---------------------------------------------------------------------------
+
+def _causal(scores):
+    nb = scores.shape[-1]
+    scores[..., np.triu_indices(nb, 1)[0], np.triu_indices(nb, 1)[1]] = -np.inf
+    return scores
+
+
+@pytest.mark.parametrize("seed", range(4))
+@pytest.mark.parametrize("group,k,w,ns", [(2, 2, 1, 0), (3, 3, 2, 1), (4, 1, 1, 1), (2, 0, 1, 0)])
+def test_group_select_matches_brute_force(seed, group, k, w, ns):
+    """Brute force on the exact (Fraction) sum of the heads' fp32-representable
+    scores; with integer scores the sum is exact in every precision."""
+    nb, kvh = 7, 2
+    g = np.random.default_rng(100 + seed)
+    if seed % 2:
+        scores = g.integers(-2, 3, size=(1, kvh * group, nb, nb)).astype(np.float64)
+    else:
+        scores = np.round(g.standard_normal((1, kvh * group, nb, nb)) * 64) / 64  # exact in fp32
+    _causal(scores)
+    idx, cnt = oracle.select_blocks_group(scores, group, k, w, ns)
+    for u in range(kvh):
+        for i in range(nb):
+            heads = range(u * group, (u + 1) * group)
+            summed = [float(sum(Fraction(float(scores[0, h, i, j])) for h in heads)) if j <= i else -np.inf
+                      for j in range(nb)]
+            expect = brute_force_select(np.array(summed), i, k, w, ns)
+            for h in heads:
+                got = list(idx[0, h, i, :cnt[0, h, i]])
+                assert got == expect, (u, h, i, got, expect)
+
+
+def test_group_of_one_is_the_per_head_rule():
+    g = np.random.default_rng(7)
+    scores = _causal(g.standard_normal((2, 3, 9, 9)))
+    a = oracle.select_blocks(scores, 3, 2, 1)
+    b = oracle.select_blocks_group(scores, 1, 3, 2, 1)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_group_of_identical_heads_keeps_each_heads_own_list():
+    g = np.random.default_rng(8)
+    one = _causal(g.standard_normal((1, 1, 10, 10)))
+    scores = np.repeat(one, 4, axis=1)  # four identical query heads sharing a KV head
+    own = oracle.select_blocks(one, 4, 1, 1)
+    grp = oracle.select_blocks_group(scores, 4, 4, 1, 1)
+    for h in range(4):
+        assert np.array_equal(grp[0][0, h], own[0][0, 0])
+        assert np.array_equal(grp[1][0, h], own[1][0, 0])
+
+
+def test_group_select_counts_follow_the_closed_form():
+    nb, group, k, w, ns = 16, 4, 5, 2, 1
+    g = np.random.default_rng(9)
+    scores = _causal(g.standard_normal((1, 8, nb, nb)))
+    idx, cnt = oracle.select_blocks_group(scores, group, k, w, ns)
+    for i in range(nb):
+        forced = set(range(max(0, i - w + 1), i + 1)) | set(range(min(ns, i + 1)))
+        assert np.all(cnt[0, :, i] == min(i + 1, k + len(forced)))
+    assert int(cnt.sum()) == 8 * sum(min(i + 1, k + w + ns) for i in range(nb))
