@@ -24,9 +24,9 @@ class BlockSparseAttention:
     def __init__(self, B_: int, Hq: int, Hkv: int, N: int, d: int, block: int, k_free: int = 0,
                  k_per_head: Optional[Sequence[int]] = None, local_window: int = 1,
                  n_sink: int = 0, scale: float = 0.0, attn_kernel: int = B.DSA_ATTN_AUTO,
-                 device=None, stream=None):
+                 select_mode: int = B.DSA_SELECT_TOPK, device=None, stream=None):
         self.params = B.Params(B_, Hq, Hkv, N, d, block, k_free, k_per_head, local_window, n_sink,
-                               scale, attn_kernel)
+                               scale, attn_kernel, select_mode)
         self.shape = (B_, Hq, Hkv, N, d, block)
         self.device = torch.device(device) if device is not None else torch.device("cuda")
         self.ws_bytes = B.dsa_workspace_size(self.params)
@@ -36,10 +36,11 @@ class BlockSparseAttention:
         B.dsa_workspace_init(self.ws, self.ws_bytes, stream)
 
     @classmethod
-    def from_workload(cls, w, k_per_head=None, attn_kernel=B.DSA_ATTN_AUTO, device=None, **over):
+    def from_workload(cls, w, k_per_head=None, attn_kernel=B.DSA_ATTN_AUTO, device=None,
+                      select_mode=B.DSA_SELECT_TOPK, **over):
         kw = dict(B_=w.B, Hq=w.Hq, Hkv=w.Hkv, N=w.N, d=w.d, block=w.block, k_free=w.k_free,
                   k_per_head=k_per_head, local_window=w.local_window, n_sink=w.n_sink,
-                  scale=w.scale, attn_kernel=attn_kernel, device=device)
+                  scale=w.scale, attn_kernel=attn_kernel, select_mode=select_mode, device=device)
         kw.update(over)
         return cls(**kw)
 

@@ -34,6 +34,10 @@ DSA_ATTN_AUTO = 0
 DSA_ATTN_TCGEN05 = 1
 DSA_ATTN_MMA_SYNC = 2
 
+# dsa_select_mode values
+DSA_SELECT_TOPK = 0
+DSA_SELECT_GROUP_TOPK = 1
+
 # Every function the header declares, with its C signature.
 _vp, _sz, _i32p, _f32p = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p
 
@@ -43,7 +47,8 @@ class dsa_params(ctypes.Structure):
                 ("N", ctypes.c_int), ("d", ctypes.c_int), ("block", ctypes.c_int),
                 ("k_free", ctypes.c_int), ("k_per_head", ctypes.POINTER(ctypes.c_int32)),
                 ("local_window", ctypes.c_int), ("n_sink", ctypes.c_int),
-                ("scale", ctypes.c_float), ("attn_kernel", ctypes.c_int)]
+                ("scale", ctypes.c_float), ("attn_kernel", ctypes.c_int),
+                ("select_mode", ctypes.c_int), ("select_tau", ctypes.c_float)]
 
 
 _P = ctypes.POINTER(dsa_params)
@@ -80,20 +85,23 @@ class Params:
     """Python-side holder of a dsa_params struct (keeps k_per_head alive)."""
 
     def __init__(self, B, Hq, Hkv, N, d, block, k_free=0, k_per_head: Optional[Sequence[int]] = None,
-                 local_window=1, n_sink=0, scale=0.0, attn_kernel=DSA_ATTN_AUTO):
+                 local_window=1, n_sink=0, scale=0.0, attn_kernel=DSA_ATTN_AUTO,
+                 select_mode=DSA_SELECT_TOPK, select_tau=0.0):
         self._kph = None
         kph_ptr = None
         if k_per_head is not None:
             self._kph = (ctypes.c_int32 * len(k_per_head))(*[int(x) for x in k_per_head])
             kph_ptr = ctypes.cast(self._kph, ctypes.POINTER(ctypes.c_int32))
         self.c = dsa_params(int(B), int(Hq), int(Hkv), int(N), int(d), int(block), int(k_free),
-                            kph_ptr, int(local_window), int(n_sink), float(scale), int(attn_kernel))
+                            kph_ptr, int(local_window), int(n_sink), float(scale), int(attn_kernel),
+                            int(select_mode), float(select_tau))
 
     @classmethod
-    def from_workload(cls, w, k_per_head=None, attn_kernel=DSA_ATTN_AUTO, **over):
+    def from_workload(cls, w, k_per_head=None, attn_kernel=DSA_ATTN_AUTO, select_mode=DSA_SELECT_TOPK,
+                      **over):
         kw = dict(B=w.B, Hq=w.Hq, Hkv=w.Hkv, N=w.N, d=w.d, block=w.block, k_free=w.k_free,
                   k_per_head=k_per_head, local_window=w.local_window, n_sink=w.n_sink,
-                  scale=w.scale, attn_kernel=attn_kernel)
+                  scale=w.scale, attn_kernel=attn_kernel, select_mode=select_mode)
         kw.update(over)
         return cls(**kw)
 

@@ -31,6 +31,10 @@ dsa_status make_shape(const dsa_params* p, Shape* s) {
   if (!std::isfinite(p->scale) || p->scale < 0.f) return DSA_ERR_INVALID_ARG;
   if (p->attn_kernel < DSA_ATTN_AUTO || p->attn_kernel > DSA_ATTN_MMA_SYNC)
     return DSA_ERR_INVALID_ARG;
+  if (p->select_mode < DSA_SELECT_TOPK || p->select_mode > DSA_SELECT_GROUP_TOPK ||
+      p->select_tau != 0.f)
+    return DSA_ERR_INVALID_ARG;
+  if (p->select_mode == DSA_SELECT_GROUP_TOPK && p->k_per_head != nullptr) return DSA_ERR_INVALID_ARG;
   long long kmax_head = 0;
   if (p->k_per_head != nullptr) {
     if (p->Hq > dsa::kMaxHeads) return DSA_ERR_UNSUPPORTED;
@@ -45,6 +49,7 @@ dsa_status make_shape(const dsa_params* p, Shape* s) {
   if (p->d != 64 && p->d != 128) return DSA_ERR_UNSUPPORTED;
   if (p->block != 32 && p->block != 64 && p->block != 128) return DSA_ERR_UNSUPPORTED;
   if (p->N % p->block != 0) return DSA_ERR_UNSUPPORTED;
+  if (p->select_mode == DSA_SELECT_GROUP_TOPK && p->Hq / p->Hkv > 32) return DSA_ERR_UNSUPPORTED;
   const int nb = p->N / p->block;
   if (nb > dsa::kMaxBlocks) return DSA_ERR_UNSUPPORTED;
   // element counts must stay well inside 64-bit and the grids inside 2^31
@@ -66,6 +71,7 @@ dsa_status make_shape(const dsa_params* p, Shape* s) {
   s->scale = p->scale == 0.f ? 1.0f / std::sqrt((float)p->d) : p->scale;
   s->kmax_head = (int)(kmax_head < nb ? kmax_head : nb);
   s->per_head = p->k_per_head != nullptr;
+  s->group_select = p->select_mode == DSA_SELECT_GROUP_TOPK;
   return DSA_OK;
 }
 

@@ -32,6 +32,7 @@ struct Shape {
   float scale;
   int kmax_head;
   bool per_head;
+  bool group_select;  // DSA_SELECT_GROUP_TOPK: one list per KV head, copied to its query heads
 };
 
 // Per-head top-k budgets passed by value to the kernels.

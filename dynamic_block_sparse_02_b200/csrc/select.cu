@@ -100,8 +100,9 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
 // ---------------------------------------------------------------------------
 // Step 3: selection of one row (b, h, i) by one warp.
 // s: the row's scores s[0..i] (shared memory); hist: 256 words of per-warp
-// scratch. Writes idx_row[0..W) (kept blocks ascending, then -1) and *cnt_out.
-// TMAX >= ceil((i+1)/32) bounds the blocks per lane.
+// scratch. Writes the list to n_out output rows u = 0..n_out-1:
+// idx_row[u * idx_stride + 0..W) (kept blocks ascending, then -1) and
+// cnt_out[u * cnt_stride]. TMAX >= ceil((i+1)/32) bounds the blocks per lane.
 //
 // Candidates are the causal blocks outside the forced set; lane l owns blocks
 // l, l+32, l+64, ..., whose order-preserving keys it keeps in registers. The k
@@ -120,8 +121,8 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
 // ---------------------------------------------------------------------------
 template <int TMAX>
 __device__ void select_row(const float* s, uint32_t* hist, int i, int k, int lw, int ns, int W,
-                           int32_t* __restrict__ idx_row, int32_t* __restrict__ cnt_out,
-                           WsHeader* hdr, int lane) {
+                           int32_t* __restrict__ idx_row, int32_t* __restrict__ cnt_out, int n_out,
+                           size_t idx_stride, size_t cnt_stride, WsHeader* hdr, int lane) {
   const int n = i + 1;
   const int win_lo = lw > 0 ? max(0, i - lw + 1) : n;  // window = [win_lo, i]
   const int nforced = (n - win_lo) + min(ns, win_lo);
@@ -263,13 +264,18 @@ __device__ void select_row(const float* s, uint32_t* hist, int i, int k, int lw,
     const uint32_t sm = __ballot_sync(kFull, sel);
     const int pos = base + __popc(sm & lt);
     if (sel) {
-      if (pos < W) idx_row[pos] = j;
-      else raise_error(hdr, DSA_ERR_DEVICE_BOUNDS, kKernSelect, i, pos);
+      if (pos < W) {
+        for (int u = 0; u < n_out; ++u) idx_row[u * idx_stride + pos] = j;
+      } else {
+        raise_error(hdr, DSA_ERR_DEVICE_BOUNDS, kKernSelect, i, pos);
+      }
     }
     base += __popc(sm);
   }
-  for (int p = base + lane; p < W; p += 32) idx_row[p] = -1;
-  if (lane == 0) *cnt_out = min(base, W);
+  for (int u = 0; u < n_out; ++u) {
+    for (int p = base + lane; p < W; p += 32) idx_row[u * idx_stride + p] = -1;
+    if (lane == 0) cnt_out[u * cnt_stride] = min(base, W);
+  }
   __syncwarp();
 }
 
@@ -428,6 +434,26 @@ score_kernel(Shape s, KBudget kb, int HB, int RB, const float* __restrict__ qp,
   __syncthreads();  // all scores written; qs/ks are free for the selection scratch
 
   const int warp = tid / 32, lane = tid % 32;
+  if (FUSED && s.group_select) {
+    // one list per query block of the tile: the tile holds every head of the
+    // KV group (rows u * RB + ii); their scores are added in head order into
+    // the first head's row, and the list goes to all of them
+    for (int ii = warp; ii < RB; ii += kSelWarps) {
+      const int i = tile.i0 + ii;
+      if (i >= i_end) continue;
+      float* const row0 = sc + ii * s.nb;
+      for (int j = lane; j <= i; j += 32) {
+        float a = row0[j];
+        for (int u = 1; u < HB; ++u) a = __fadd_rn(a, sc[(u * RB + ii) * s.nb + j]);
+        row0[j] = a;
+      }
+      __syncwarp();
+      const size_t row = ((size_t)tile.b * s.Hq + tile.h0) * s.nb + i;
+      select_row<TMAX>(row0, sk + warp * kHistWords, i, kb.k[0], s.lw, s.ns, s.W, idx + row * s.W,
+                       cnt + row, HB, (size_t)s.nb * s.W, (size_t)s.nb, hdr, lane);
+    }
+    return;
+  }
   for (int r = warp; r < kRowTile; r += kSelWarps) {
     const int h = tile.h0 + r / RB, i = tile.i0 + r % RB;
     if (r >= HB * RB || h >= h_end || i >= i_end) continue;
@@ -435,7 +461,7 @@ score_kernel(Shape s, KBudget kb, int HB, int RB, const float* __restrict__ qp,
     if (FUSED) {
       const int k = s.per_head ? kb.k[h] : kb.k[0];
       select_row<TMAX>(sc + r * s.nb, sk + warp * kHistWords, i, k, s.lw, s.ns, s.W, idx + row * s.W,
-                       cnt + row, hdr, lane);
+                       cnt + row, 1, 0, 0, hdr, lane);
     } else {
       float* dst = scores + row * s.nb;
       for (int j = lane; j < s.nb; j += 32) dst[j] = (j <= i) ? sc[r * s.nb + j] : -INFINITY;
@@ -443,7 +469,9 @@ score_kernel(Shape s, KBudget kb, int HB, int RB, const float* __restrict__ qp,
   }
 }
 
-// Selection on caller scores: one warp per row (b, h, i).
+// Selection on caller scores: one warp per row (b, h, i), or with the
+// group-shared rule per (b, KV head, i) from the group's scores added in head
+// order (the same fp32 additions as the fused kernel).
 template <int TMAX>
 __global__ void __launch_bounds__(kSelThreads)
 select_kernel(Shape s, KBudget kb, const float* __restrict__ scores, int32_t* __restrict__ idx,
@@ -453,14 +481,29 @@ select_kernel(Shape s, KBudget kb, const float* __restrict__ scores, int32_t* __
   const long long row = (long long)blockIdx.x * kSelWarps + warp;
   if (row >= n_rows) return;
   const int i = (int)(row % s.nb);
-  const int h = (int)((row / s.nb) % s.Hq);
   float* sc = sm_f + warp * s.nb;
   uint32_t* sk = reinterpret_cast<uint32_t*>(sm_f + kSelWarps * s.nb) + warp * kHistWords;
+  if (s.group_select) {
+    const long long bk = row / s.nb;  // b * Hkv + KV head
+    const size_t head0 = (size_t)bk * s.group;  // b * Hq + first query head of the group
+    for (int j = lane; j <= i; j += 32) {
+      float a = scores[(head0 * s.nb + i) * s.nb + j];
+      for (int u = 1; u < s.group; ++u) a = __fadd_rn(a, scores[((head0 + u) * s.nb + i) * s.nb + j]);
+      sc[j] = a;
+    }
+    __syncwarp();
+    const size_t out = head0 * s.nb + i;
+    select_row<TMAX>(sc, sk, i, kb.k[0], s.lw, s.ns, s.W, idx + out * s.W, cnt + out, s.group,
+                     (size_t)s.nb * s.W, (size_t)s.nb, hdr, lane);
+    return;
+  }
+  const int h = (int)((row / s.nb) % s.Hq);
   const float* src = scores + (size_t)row * s.nb;
   for (int j = lane; j <= i; j += 32) sc[j] = src[j];
   __syncwarp();
   const int k = s.per_head ? kb.k[h] : kb.k[0];
-  select_row<TMAX>(sc, sk, i, k, s.lw, s.ns, s.W, idx + (size_t)row * s.W, cnt + row, hdr, lane);
+  select_row<TMAX>(sc, sk, i, k, s.lw, s.ns, s.W, idx + (size_t)row * s.W, cnt + row, 1, 0, 0, hdr,
+                   lane);
 }
 
 void row_tiling(const Shape& s, int& HB, int& RB) {
@@ -534,7 +577,7 @@ cudaError_t launch_score_select(const Shape& s, const KBudget& kb, const float* 
 
 cudaError_t launch_select(const Shape& s, const KBudget& kb, const float* scores, int32_t* idx,
                           int32_t* cnt, WsHeader* hdr, cudaStream_t st) {
-  const long long n_rows = (long long)s.B * s.Hq * s.nb;
+  const long long n_rows = (long long)s.B * (s.group_select ? s.Hkv : s.Hq) * s.nb;
   const long long grid = (n_rows + kSelWarps - 1) / kSelWarps;
   const size_t smem = (size_t)kSelWarps * (s.nb + kHistWords) * sizeof(float);
   auto f = select_tmax(s.nb) == 8 ? select_kernel<8> : select_tmax(s.nb) == 16 ? select_kernel<16> : select_kernel<32>;

@@ -68,6 +68,17 @@ typedef enum dsa_status {
   DSA_ERR_DEVICE_BOUNDS = 6   /* a kernel met an index outside its valid range (device flag) */
 } dsa_status;
 
+/* Selection rule (dsa_params.select_mode). */
+typedef enum dsa_select_mode {
+  DSA_SELECT_TOPK = 0,       /* per (batch, query head, query block): forced + top-k (steps 1-3 above) */
+  DSA_SELECT_GROUP_TOPK = 1  /* per (batch, KV head, query block): the same rule on the sum of the
+                                group's query-head scores s_h (fp32, added in head order); every
+                                query head of the group receives that list. The pages note that
+                                GQA's shared KV cache makes one index per KV head natural
+                                (zblog.xzdbk.com/559 post, section on speculative decoding) and
+                                merge the lists of several index heads (DSA post, section 2.1). */
+} dsa_select_mode;
+
 /* Attention kernel choice (dsa_params.attn_kernel). */
 typedef enum dsa_attn_kernel {
   DSA_ATTN_AUTO = 0,     /* the fastest kernel this library has for the shape */
@@ -90,6 +101,9 @@ typedef enum dsa_attn_kernel {
  *   n_sink           : >= 0; forces blocks {0 .. n_sink-1}.
  *   scale            : softmax scale; 0 means 1/sqrt(d); must be finite, >= 0.
  *   attn_kernel      : a dsa_attn_kernel value.
+ *   select_mode      : a dsa_select_mode value. DSA_SELECT_GROUP_TOPK needs
+ *                      k_per_head == NULL and Hq/Hkv <= 32.
+ *   select_tau       : reserved, must be 0.
  */
 typedef struct dsa_params {
   int B, Hq, Hkv, N, d;
@@ -100,6 +114,8 @@ typedef struct dsa_params {
   int n_sink;
   float scale;
   int attn_kernel;
+  int select_mode;
+  float select_tau;
 } dsa_params;
 
 /* Row width W of idx: min(nb, max_h k_h + local_window + n_sink). 0 for an

@@ -139,3 +139,18 @@ def test_empty_problems_return_ok_without_touching_pointers():
         assert status_of_forward(p, q=None, k=None, v=None, out=None, ws=None) == B.DSA_OK
         assert B.dsa_workspace_size(p) == 256
         assert B.dsa_kmax(p) == 0
+
+
+def test_select_mode_checks():
+    base = dict(B=1, Hq=8, Hkv=2, N=1024, d=64, block=64, k_free=4, local_window=1, n_sink=1)
+    assert status_of_forward(B.Params(**base, select_mode=7)) == B.DSA_ERR_INVALID_ARG
+    assert status_of_forward(B.Params(**base, select_mode=-1)) == B.DSA_ERR_INVALID_ARG
+    assert status_of_forward(B.Params(**base, select_tau=0.5)) == B.DSA_ERR_INVALID_ARG
+    # the group rule shares one budget per KV head
+    assert status_of_forward(B.Params(**base, k_per_head=[1] * 8, select_mode=B.DSA_SELECT_GROUP_TOPK)) \
+        == B.DSA_ERR_INVALID_ARG
+    big = dict(base, Hq=66, Hkv=1)
+    assert status_of_forward(B.Params(**big, select_mode=B.DSA_SELECT_GROUP_TOPK)) == B.DSA_ERR_UNSUPPORTED
+    ok = B.Params(**base, select_mode=B.DSA_SELECT_GROUP_TOPK)
+    assert B.dsa_kmax(ok) == B.dsa_kmax(B.Params(**base))
+    assert B.dsa_workspace_size(ok) == B.dsa_workspace_size(B.Params(**base))
