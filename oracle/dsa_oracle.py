@@ -24,6 +24,9 @@ What is computed, and where the pages say so:
 * Group-shared selection (an alternative rule): one list per KV head, chosen
   by the same rule from the sum of its query heads' block scores and used by
   all of them (see group_scores).
+* Threshold selection (an alternative rule): forced blocks plus the blocks
+  whose share of the softmax over the row's block logits reaches tau, at most
+  k of them (see select_blocks_threshold).
 * Attention. softmax(Q K^T * scale) V over the kept key blocks only, with the
   causal mask inside the diagonal block ("稀疏注意力 vs Flash Attention v2",
   section 1 pseudocode: scores, then the sparsity pattern, then softmax with
@@ -203,6 +206,74 @@ def select_blocks_group(scores: np.ndarray, group: int, k_free: int, local_windo
     idx = np.repeat(idx_g, group, axis=1)
     cnt = np.repeat(cnt_g, group, axis=1)
     return idx, cnt
+
+
+def block_probabilities(scores_row: np.ndarray, i: int, scale: float) -> np.ndarray:
+    """Softmax over the causal key blocks 0..i of one query block's logits
+    scale * s(i, j), in fp64 (the block-level attention distribution that the
+    threshold rule compares with tau)."""
+    z = scale * np.asarray(scores_row[:i + 1], dtype=np.float64)
+    e = np.exp(z - z.max())
+    return e / e.sum()
+
+
+def select_blocks_threshold(scores: np.ndarray, tau: float, k_free, local_window: int,
+                            n_sink: int, scale: float,
+                            width: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Threshold selection: the forced set plus every remaining causal block
+    whose block probability (block_probabilities) is >= tau, at most k_free of
+    them (the best by the top-k order when more pass).
+
+    Follows the DeepSeek NSA article, section 2.2 (block_sparsify with a
+    threshold on the fp32 scores, 0.1 there) and section 4.2 (start the
+    threshold at 0.05), and the zblog post's adaptive k-or-threshold advice
+    (section 模型精度与稀疏度的动态平衡). The pages do not say what the
+    threshold is compared with; the plain reading used here is each block's
+    share of the softmax over the row's causal block logits.
+    """
+    B, Hq, nb, _ = scores.shape
+    ks = np.full(Hq, int(k_free), dtype=np.int64) if np.isscalar(k_free) else \
+        np.asarray(k_free, dtype=np.int64)
+    if width is None:
+        width = row_width(nb, int(ks.max()) if Hq else 0, local_window, n_sink)
+    keff = np.zeros((B, Hq, nb), dtype=np.int64)
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(nb):
+                forced = forced_set(i, local_window, n_sink)
+                p = block_probabilities(scores[b, h, i], i, scale)
+                passing = sum(1 for j in range(i + 1) if j not in forced and p[j] >= tau)
+                keff[b, h, i] = min(int(ks[h]), passing)
+    idx = np.full((B, Hq, nb, width), -1, dtype=np.int32)
+    cnt = np.zeros((B, Hq, nb), dtype=np.int32)
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(nb):
+                # the ranking of select_blocks on this row, with the row's own budget
+                idx[b, h, i], cnt[b, h, i] = _select_row(scores[b, h, i], i, int(keff[b, h, i]),
+                                                         local_window, n_sink, width)
+    return idx, cnt
+
+
+def _select_row(scores_row: np.ndarray, i: int, k: int, local_window: int, n_sink: int,
+                width: int) -> Tuple[np.ndarray, int]:
+    """select_blocks for one row with budget k: forced set plus the k best
+    candidates by fp32 score, ties to the lower index; ascending, -1 padded."""
+    forced = forced_set(i, local_window, n_sink)
+    cand = np.array([j for j in range(i + 1) if j not in forced], dtype=np.int64)
+    take = min(k, cand.size)
+    s32 = np.asarray(scores_row, dtype=np.float64).astype(np.float32)
+    if take > 0:
+        order = np.lexsort((cand, -s32[cand].astype(np.float64)))
+        picks = cand[order[:take]]
+    else:
+        picks = np.empty(0, dtype=np.int64)
+    kept = sorted(forced | set(int(j) for j in picks))
+    if len(kept) > width:
+        raise ValueError("row width too small for the kept set")
+    out = np.full(width, -1, dtype=np.int32)
+    out[:len(kept)] = kept
+    return out, len(kept)
 
 
 # ---------------------------------------------------------------------------

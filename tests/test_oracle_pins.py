@@ -432,3 +432,56 @@ def test_group_select_counts_follow_the_closed_form():
         forced = set(range(max(0, i - w + 1), i + 1)) | set(range(min(ns, i + 1)))
         assert np.all(cnt[0, :, i] == min(i + 1, k + len(forced)))
     assert int(cnt.sum()) == 8 * sum(min(i + 1, k + w + ns) for i in range(nb))
+
+
+# ---------------------------------------------------------------------------
+# Threshold selection (block probability >= tau, at most k)
+# ---------------------------------------------------------------------------
+
+def test_threshold_worked_example():
+    """Row 3 with logits ln 1, ln 2, ln 3, ln 4: block probabilities 0.1, 0.2,
+    0.3, 0.4; block 3 is the forced diagonal."""
+    nb = 4
+    scores = _causal(np.zeros((1, 1, nb, nb)))
+    scores[0, 0, 3, :4] = np.log([1.0, 2.0, 3.0, 4.0])
+    p = oracle.block_probabilities(scores[0, 0, 3], 3, 1.0)
+    np.testing.assert_allclose(p, [0.1, 0.2, 0.3, 0.4], rtol=1e-14)
+    row = lambda tau, k: list(oracle.select_blocks_threshold(scores, tau, k, 1, 0, 1.0)[0][0, 0, 3])
+    assert row(0.15, 5)[:3] == [1, 2, 3]      # 0.2 and 0.3 pass
+    assert row(0.15, 1)[:2] == [2, 3]         # cap at k: the better of the two
+    assert row(0.25, 5)[:2] == [2, 3]         # only 0.3 passes
+    assert row(0.35, 5)[:1] == [3]            # none pass: the forced block alone
+    assert row(0.05, 5)[:4] == [0, 1, 2, 3]   # all pass
+
+
+def test_threshold_limits_reduce_to_top_k():
+    g = np.random.default_rng(11)
+    scores = _causal(g.standard_normal((1, 2, 12, 12)))
+    for k in (0, 2, 5):
+        lo = oracle.select_blocks_threshold(scores, 1e-300, k, 2, 1, 0.5)
+        ref = oracle.select_blocks(scores, k, 2, 1)
+        assert np.array_equal(lo[0], ref[0]) and np.array_equal(lo[1], ref[1])
+        hi = oracle.select_blocks_threshold(scores, 1.5, k, 2, 1, 0.5)
+        none = oracle.select_blocks(scores, 0, 2, 1, width=ref[0].shape[-1])
+        assert np.array_equal(hi[0], none[0]) and np.array_equal(hi[1], none[1])
+
+
+@pytest.mark.parametrize("seed", range(4))
+@pytest.mark.parametrize("tau,k,w,ns,scale", [(0.1, 3, 1, 0, 1.0), (0.05, 2, 2, 1, 0.7),
+                                              (0.2, 8, 1, 1, 2.0), (0.01, 1, 0, 2, 1.3)])
+def test_threshold_matches_brute_force(seed, tau, k, w, ns, scale):
+    nb = 8
+    g = np.random.default_rng(200 + seed)
+    scores = _causal(g.standard_normal((1, 1, nb, nb)) * 1.5)
+    idx, cnt = oracle.select_blocks_threshold(scores, tau, k, w, ns, scale)
+    s32 = scores.astype(np.float32)
+    for i in range(nb):
+        logits = [scale * float(scores[0, 0, i, j]) for j in range(i + 1)]
+        mx = max(logits)
+        e = [math.exp(v - mx) for v in logits]
+        z = math.fsum(e)
+        forced = set(range(max(0, i - w + 1), i + 1)) if w > 0 else set()
+        forced |= set(range(min(ns, i + 1)))
+        passing = [j for j in range(i + 1) if j not in forced and e[j] / z >= tau]
+        expect = brute_force_select(s32[0, 0, i], i, min(k, len(passing)), w, ns)
+        assert list(idx[0, 0, i, :cnt[0, 0, i]]) == expect, (i, passing)
