@@ -24,9 +24,10 @@ class BlockSparseAttention:
     def __init__(self, B_: int, Hq: int, Hkv: int, N: int, d: int, block: int, k_free: int = 0,
                  k_per_head: Optional[Sequence[int]] = None, local_window: int = 1,
                  n_sink: int = 0, scale: float = 0.0, attn_kernel: int = B.DSA_ATTN_AUTO,
-                 select_mode: int = B.DSA_SELECT_TOPK, device=None, stream=None):
+                 select_mode: int = B.DSA_SELECT_TOPK, select_tau: float = 0.0, device=None,
+                 stream=None):
         self.params = B.Params(B_, Hq, Hkv, N, d, block, k_free, k_per_head, local_window, n_sink,
-                               scale, attn_kernel, select_mode)
+                               scale, attn_kernel, select_mode, select_tau)
         self.shape = (B_, Hq, Hkv, N, d, block)
         self.device = torch.device(device) if device is not None else torch.device("cuda")
         self.ws_bytes = B.dsa_workspace_size(self.params)

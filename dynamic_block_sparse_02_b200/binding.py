@@ -37,6 +37,7 @@ DSA_ATTN_MMA_SYNC = 2
 # dsa_select_mode values
 DSA_SELECT_TOPK = 0
 DSA_SELECT_GROUP_TOPK = 1
+DSA_SELECT_THRESHOLD = 2
 
 # Every function the header declares, with its C signature.
 _vp, _sz, _i32p, _f32p = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p

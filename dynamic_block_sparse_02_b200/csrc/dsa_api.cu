@@ -31,8 +31,11 @@ dsa_status make_shape(const dsa_params* p, Shape* s) {
   if (!std::isfinite(p->scale) || p->scale < 0.f) return DSA_ERR_INVALID_ARG;
   if (p->attn_kernel < DSA_ATTN_AUTO || p->attn_kernel > DSA_ATTN_MMA_SYNC)
     return DSA_ERR_INVALID_ARG;
-  if (p->select_mode < DSA_SELECT_TOPK || p->select_mode > DSA_SELECT_GROUP_TOPK ||
-      p->select_tau != 0.f)
+  if (p->select_mode < DSA_SELECT_TOPK || p->select_mode > DSA_SELECT_THRESHOLD)
+    return DSA_ERR_INVALID_ARG;
+  if (p->select_mode == DSA_SELECT_THRESHOLD
+          ? !(p->select_tau > 0.f && p->select_tau <= 1.f)
+          : p->select_tau != 0.f)
     return DSA_ERR_INVALID_ARG;
   if (p->select_mode == DSA_SELECT_GROUP_TOPK && p->k_per_head != nullptr) return DSA_ERR_INVALID_ARG;
   long long kmax_head = 0;
@@ -72,6 +75,8 @@ dsa_status make_shape(const dsa_params* p, Shape* s) {
   s->kmax_head = (int)(kmax_head < nb ? kmax_head : nb);
   s->per_head = p->k_per_head != nullptr;
   s->group_select = p->select_mode == DSA_SELECT_GROUP_TOPK;
+  s->tau = p->select_mode == DSA_SELECT_THRESHOLD ? p->select_tau : 0.f;
+  s->c2 = s->scale * 1.4426950408889634f;
   return DSA_OK;
 }
 

@@ -33,6 +33,8 @@ struct Shape {
   int kmax_head;
   bool per_head;
   bool group_select;  // DSA_SELECT_GROUP_TOPK: one list per KV head, copied to its query heads
+  float tau;          // DSA_SELECT_THRESHOLD: tau (0 in the other modes)
+  float c2;           // scale * log2(e): block logits in base 2
 };
 
 // Per-head top-k budgets passed by value to the kernels.

@@ -121,15 +121,51 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
 // ---------------------------------------------------------------------------
 template <int TMAX>
 __device__ void select_row(const float* s, uint32_t* hist, int i, int k, int lw, int ns, int W,
-                           int32_t* __restrict__ idx_row, int32_t* __restrict__ cnt_out, int n_out,
-                           size_t idx_stride, size_t cnt_stride, WsHeader* hdr, int lane) {
+                           float tau, float c2, int32_t* __restrict__ idx_row,
+                           int32_t* __restrict__ cnt_out, int n_out, size_t idx_stride,
+                           size_t cnt_stride, WsHeader* hdr, int lane) {
   const int n = i + 1;
   const int win_lo = lw > 0 ? max(0, i - lw + 1) : n;  // window = [win_lo, i]
   const int nforced = (n - win_lo) + min(ns, win_lo);
   const int ncand = n - nforced;
-  const int keff = min(k, ncand);
   const int T = (n + 31) >> 5;
   const uint32_t lt = (1u << lane) - 1u;
+
+  // Threshold rule (tau > 0): the budget shrinks to the candidates whose block
+  // probability 2^(c2 (s_j - m)) / Z over the causal blocks reaches tau. The
+  // passing candidates are the highest-scoring ones, so the top-k machinery
+  // below then keeps exactly them (or the best k when more pass).
+  if (tau > 0.f) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) {
+      if (t >= T) break;
+      const int j = t * 32 + lane;
+      if (j < n) m = fmaxf(m, s[j]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+    float z = 0.f;
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) {
+      if (t >= T) break;
+      const int j = t * 32 + lane;
+      if (j < n) z += exp2f(c2 * (s[j] - m));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(kFull, z, off);
+    const float bar = tau * z;
+    int passing = 0;
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) {
+      if (t >= T) break;
+      const int j = t * 32 + lane;
+      const bool pass = j >= ns && j < win_lo && exp2f(c2 * (s[j] - m)) >= bar;
+      passing += __popc(__ballot_sync(kFull, pass));
+    }
+    k = min(k, passing);
+  }
+  const int keff = min(k, ncand);
 
   // candidates are ns <= j < win_lo (the forced blocks are j < ns and j >= win_lo)
   uint32_t key[TMAX];  // 0: not a candidate (every finite score has a key >= 0x00800000)
@@ -449,8 +485,8 @@ score_kernel(Shape s, KBudget kb, int HB, int RB, const float* __restrict__ qp,
       }
       __syncwarp();
       const size_t row = ((size_t)tile.b * s.Hq + tile.h0) * s.nb + i;
-      select_row<TMAX>(row0, sk + warp * kHistWords, i, kb.k[0], s.lw, s.ns, s.W, idx + row * s.W,
-                       cnt + row, HB, (size_t)s.nb * s.W, (size_t)s.nb, hdr, lane);
+      select_row<TMAX>(row0, sk + warp * kHistWords, i, kb.k[0], s.lw, s.ns, s.W, s.tau, s.c2,
+                       idx + row * s.W, cnt + row, HB, (size_t)s.nb * s.W, (size_t)s.nb, hdr, lane);
     }
     return;
   }
@@ -460,8 +496,8 @@ score_kernel(Shape s, KBudget kb, int HB, int RB, const float* __restrict__ qp,
     const size_t row = ((size_t)tile.b * s.Hq + h) * s.nb + i;
     if (FUSED) {
       const int k = s.per_head ? kb.k[h] : kb.k[0];
-      select_row<TMAX>(sc + r * s.nb, sk + warp * kHistWords, i, k, s.lw, s.ns, s.W, idx + row * s.W,
-                       cnt + row, 1, 0, 0, hdr, lane);
+      select_row<TMAX>(sc + r * s.nb, sk + warp * kHistWords, i, k, s.lw, s.ns, s.W, s.tau, s.c2,
+                       idx + row * s.W, cnt + row, 1, 0, 0, hdr, lane);
     } else {
       float* dst = scores + row * s.nb;
       for (int j = lane; j < s.nb; j += 32) dst[j] = (j <= i) ? sc[r * s.nb + j] : -INFINITY;
@@ -493,8 +529,8 @@ select_kernel(Shape s, KBudget kb, const float* __restrict__ scores, int32_t* __
     }
     __syncwarp();
     const size_t out = head0 * s.nb + i;
-    select_row<TMAX>(sc, sk, i, kb.k[0], s.lw, s.ns, s.W, idx + out * s.W, cnt + out, s.group,
-                     (size_t)s.nb * s.W, (size_t)s.nb, hdr, lane);
+    select_row<TMAX>(sc, sk, i, kb.k[0], s.lw, s.ns, s.W, s.tau, s.c2, idx + out * s.W, cnt + out,
+                     s.group, (size_t)s.nb * s.W, (size_t)s.nb, hdr, lane);
     return;
   }
   const int h = (int)((row / s.nb) % s.Hq);
@@ -502,8 +538,8 @@ select_kernel(Shape s, KBudget kb, const float* __restrict__ scores, int32_t* __
   for (int j = lane; j <= i; j += 32) sc[j] = src[j];
   __syncwarp();
   const int k = s.per_head ? kb.k[h] : kb.k[0];
-  select_row<TMAX>(sc, sk, i, k, s.lw, s.ns, s.W, idx + (size_t)row * s.W, cnt + row, 1, 0, 0, hdr,
-                   lane);
+  select_row<TMAX>(sc, sk, i, k, s.lw, s.ns, s.W, s.tau, s.c2, idx + (size_t)row * s.W, cnt + row, 1, 0,
+                   0, hdr, lane);
 }
 
 void row_tiling(const Shape& s, int& HB, int& RB) {

@@ -71,12 +71,18 @@ typedef enum dsa_status {
 /* Selection rule (dsa_params.select_mode). */
 typedef enum dsa_select_mode {
   DSA_SELECT_TOPK = 0,       /* per (batch, query head, query block): forced + top-k (steps 1-3 above) */
-  DSA_SELECT_GROUP_TOPK = 1  /* per (batch, KV head, query block): the same rule on the sum of the
+  DSA_SELECT_GROUP_TOPK = 1, /* per (batch, KV head, query block): the same rule on the sum of the
                                 group's query-head scores s_h (fp32, added in head order); every
                                 query head of the group receives that list. The pages note that
                                 GQA's shared KV cache makes one index per KV head natural
                                 (zblog.xzdbk.com/559 post, section on speculative decoding) and
                                 merge the lists of several index heads (DSA post, section 2.1). */
+  DSA_SELECT_THRESHOLD = 2   /* per (batch, query head, query block): forced + the remaining causal
+                                blocks j whose block probability softmax_j(scale * s(i, j)) over
+                                j <= i is >= select_tau, at most k of them (the best first). The
+                                DeepSeek NSA article, section 2.2, thresholds the fp32 scores
+                                (0.1), section 4.2 starts the threshold at 0.05; the zblog post
+                                adapts k or the threshold per input. */
 } dsa_select_mode;
 
 /* Attention kernel choice (dsa_params.attn_kernel). */
@@ -103,7 +109,11 @@ typedef enum dsa_attn_kernel {
  *   attn_kernel      : a dsa_attn_kernel value.
  *   select_mode      : a dsa_select_mode value. DSA_SELECT_GROUP_TOPK needs
  *                      k_per_head == NULL and Hq/Hkv <= 32.
- *   select_tau       : reserved, must be 0.
+ *   select_tau       : DSA_SELECT_THRESHOLD: the threshold tau, 0 < tau <= 1;
+ *                      other modes: must be 0. The block probabilities are
+ *                      computed in fp32 (exp2 of scale * log2(e) * (s - max)),
+ *                      so a block within ~1e-6 relative of the threshold may
+ *                      fall on either side of it.
  */
 typedef struct dsa_params {
   int B, Hq, Hkv, N, d;

@@ -151,6 +151,12 @@ def test_select_mode_checks():
         == B.DSA_ERR_INVALID_ARG
     big = dict(base, Hq=66, Hkv=1)
     assert status_of_forward(B.Params(**big, select_mode=B.DSA_SELECT_GROUP_TOPK)) == B.DSA_ERR_UNSUPPORTED
+    # the threshold rule needs 0 < tau <= 1
+    for tau in (0.0, -0.1, 1.5, float("nan")):
+        assert status_of_forward(B.Params(**base, select_mode=B.DSA_SELECT_THRESHOLD, select_tau=tau)) \
+            == B.DSA_ERR_INVALID_ARG
+    thr = B.Params(**base, select_mode=B.DSA_SELECT_THRESHOLD, select_tau=0.05)
+    assert B.dsa_kmax(thr) == B.dsa_kmax(B.Params(**base))
     ok = B.Params(**base, select_mode=B.DSA_SELECT_GROUP_TOPK)
     assert B.dsa_kmax(ok) == B.dsa_kmax(B.Params(**base))
     assert B.dsa_workspace_size(ok) == B.dsa_workspace_size(B.Params(**base))
