@@ -382,6 +382,76 @@ def forward(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, block: i
     return idx, cnt, att
 
 
+# ---------------------------------------------------------------------------
+# Decode: one new query token against a KV cache
+# ---------------------------------------------------------------------------
+
+def decode(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, length: int, block: int,
+           k_free, local_window: int, n_sink: int, scale: float = 0.0, mode: str = "topk",
+           tau: float = 0.0):
+    """One decode step: query token q [B, Hq, d] at position length-1, keys and
+    values [B, Hkv, >= length, d] (only the first ``length`` are read).
+
+    The token's query block is i = (length-1) // block. Block scores are
+    q . mean(K block j) for j <= i, the mean taken over the block's present
+    keys (all of them for j < i, the first length - i*block for j = i).
+    Selection follows the prefill rules on that single row ("topk", "group":
+    the group's query heads' scores summed, "threshold": block probability >=
+    tau, at most k); attention is softmax(q K^T * scale) V over the present keys
+    of the kept blocks (the pages: store the sparse index with the KV cache and
+    reuse it at inference, zblog.xzdbk.com/559 post, section 动态开销与计算收益的
+    权衡, point 2).
+
+    Returns idx int32 [B,Hq,W], cnt int32 [B,Hq], out fp64 [B,Hq,d], lse fp64 [B,Hq].
+    """
+    q = bf16_to_f64(q_bits)
+    k = bf16_to_f64(k_bits)
+    v = bf16_to_f64(v_bits)
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    g = Hq // Hkv
+    i = (length - 1) // block
+    nb_row = i + 1
+    if scale == 0.0:
+        scale = 1.0 / math.sqrt(d)
+    ks = np.full(Hq, int(k_free), dtype=np.int64) if np.isscalar(k_free) else \
+        np.asarray(k_free, dtype=np.int64)
+    width = row_width(k.shape[2] // block, int(ks.max()) if Hq else 0, local_window, n_sink)
+    kmeans = np.zeros((B, Hkv, nb_row, d))
+    for j in range(nb_row):
+        hi = min((j + 1) * block, length)
+        kmeans[:, :, j] = k[:, :, j * block:hi].mean(axis=2)
+    scores = np.einsum("bhd,bhjd->bhj", q, np.repeat(kmeans, g, axis=1))  # [B, Hq, i+1]
+    if mode == "group":
+        summed = scores.reshape(B, Hkv, g, nb_row).sum(axis=2)
+        scores = np.repeat(summed, g, axis=1)
+    idx = np.full((B, Hq, width), -1, dtype=np.int32)
+    cnt = np.zeros((B, Hq), dtype=np.int32)
+    out = np.zeros((B, Hq, d))
+    lse = np.full((B, Hq), -np.inf)
+    for b in range(B):
+        for h in range(Hq):
+            row = scores[b, h]
+            kk = int(ks[h])
+            if mode == "threshold":
+                forced = forced_set(i, local_window, n_sink)
+                p = block_probabilities(row, i, scale)
+                kk = min(kk, sum(1 for j in range(i + 1) if j not in forced and p[j] >= tau))
+            idx[b, h], cnt[b, h] = _select_row(row, i, kk, local_window, n_sink, width)
+            keys = np.concatenate([np.arange(j * block, min((j + 1) * block, length))
+                                   for j in idx[b, h, :cnt[b, h]]]) if cnt[b, h] else np.empty(0, int)
+            if keys.size == 0:
+                continue
+            kv = h // g
+            logits = scale * (k[b, kv, keys] @ q[b, h])
+            mx = logits.max()
+            e = np.exp(logits - mx)
+            z = e.sum()
+            out[b, h] = (e / z) @ v[b, kv, keys]
+            lse[b, h] = mx + math.log(z)
+    return idx, cnt, out, lse
+
+
 def attended_pairs(idx: np.ndarray, cnt: np.ndarray, block: int) -> int:
     """Number of (query, key) score pairs that the kept blocks make visible (causal)."""
     total = 0

@@ -485,3 +485,78 @@ def test_threshold_matches_brute_force(seed, tau, k, w, ns, scale):
         passing = [j for j in range(i + 1) if j not in forced and e[j] / z >= tau]
         expect = brute_force_select(s32[0, 0, i], i, min(k, len(passing)), w, ns)
         assert list(idx[0, 0, i, :cnt[0, 0, i]]) == expect, (i, passing)
+
+
+# ---------------------------------------------------------------------------
+# Decode (one query token against a KV cache)
+# ---------------------------------------------------------------------------
+
+def _bf16(x):
+    return W.f32_to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+def test_decode_dense_is_textbook_attention_of_the_last_token():
+    g = np.random.default_rng(41)
+    Bn, Hq, Hkv, N, d, bs, L = 2, 4, 2, 256, 16, 32, 201
+    q = _bf16(g.standard_normal((Bn, Hq, d)))
+    k = _bf16(g.standard_normal((Bn, Hkv, N, d)))
+    v = _bf16(g.standard_normal((Bn, Hkv, N, d)))
+    idx, cnt, out, lse = oracle.decode(q, k, v, L, bs, 1000, 1, 0)
+    qf, kf, vf = (W.bf16_bits_to_f32(a).astype(np.float64) for a in (q, k, v))
+    for b in range(Bn):
+        for h in range(Hq):
+            assert cnt[b, h] == (L - 1) // bs + 1
+            x = kf[b, h // 2, :L] @ qf[b, h] / math.sqrt(d)
+            p = np.exp(x - x.max())
+            np.testing.assert_allclose(out[b, h], (p / p.sum()) @ vf[b, h // 2, :L], rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(lse[b, h], x.max() + math.log(p.sum()), rtol=1e-13)
+
+
+def test_decode_matches_the_prefill_row_of_a_constant_query_block():
+    """When every row of the last query block equals q and the block is
+    complete, the block mean is q: decode keeps the prefill's row and its
+    output is the prefill output of the block's last token."""
+    g = np.random.default_rng(42)
+    Bn, Hq, Hkv, N, d, bs = 1, 4, 2, 12 * 32, 16, 32
+    k_free, w, ns = 3, 1, 1
+    L = N
+    qtok = g.standard_normal((Bn, Hq, d)).astype(np.float32)
+    Q = g.standard_normal((Bn, Hq, N, d)).astype(np.float32)
+    Q[:, :, N - bs:] = qtok[:, :, None, :]
+    K = g.standard_normal((Bn, Hkv, N, d)).astype(np.float32)
+    V = g.standard_normal((Bn, Hkv, N, d)).astype(np.float32)
+    idx_p, cnt_p, (o_p, lse_p) = oracle.forward(_bf16(Q), _bf16(K), _bf16(V), bs, k_free, w, ns)
+    idx, cnt, out, lse = oracle.decode(_bf16(qtok), _bf16(K), _bf16(V), L, bs, k_free, w, ns)
+    i = N // bs - 1
+    np.testing.assert_array_equal(idx, idx_p[:, :, i, :idx.shape[-1]])
+    np.testing.assert_array_equal(cnt, cnt_p[:, :, i])
+    np.testing.assert_allclose(out, o_p[:, :, N - 1], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(lse, lse_p[:, :, N - 1], rtol=1e-13)
+
+
+def test_decode_partial_block_uses_present_keys_only():
+    g = np.random.default_rng(43)
+    Bn, Hq, Hkv, N, d, bs, L = 1, 2, 1, 128, 8, 32, 70   # block 2 holds keys 64..69
+    q = _bf16(g.standard_normal((Bn, Hq, d)))
+    k = _bf16(g.standard_normal((Bn, Hkv, N, d)) * 3)
+    v = _bf16(g.standard_normal((Bn, Hkv, N, d)))
+    idx, cnt, out, lse = oracle.decode(q, k, v, L, bs, 0, 1, 0)   # the diagonal block only
+    assert list(idx[0, 0, :cnt[0, 0]]) == [2]
+    qf, kf, vf = (W.bf16_bits_to_f32(a).astype(np.float64) for a in (q, k, v))
+    for h in range(Hq):
+        x = kf[0, 0, 64:70] @ qf[0, h] / math.sqrt(d)
+        p = np.exp(x - x.max())
+        np.testing.assert_allclose(out[0, h], (p / p.sum()) @ vf[0, 0, 64:70], rtol=1e-12, atol=1e-14)
+
+
+def test_decode_group_of_identical_heads_equals_per_head():
+    g = np.random.default_rng(44)
+    d, bs, N, L = 16, 32, 20 * 32, 20 * 32 - 5
+    one = g.standard_normal((1, 1, d))
+    q = _bf16(np.repeat(one, 4, axis=1))
+    k = _bf16(g.standard_normal((1, 1, N, d)))
+    v = _bf16(g.standard_normal((1, 1, N, d)))
+    a = oracle.decode(q, k, v, L, bs, 4, 2, 1)
+    b = oracle.decode(q, k, v, L, bs, 4, 2, 1, mode="group")
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
