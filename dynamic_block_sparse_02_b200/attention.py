@@ -95,5 +95,25 @@ class BlockSparseAttention:
                               self.stream)
         return out
 
+    def pooled_key_cache(self):
+        """An fp32 [B, Hkv, N/block, d] buffer for the pooled key cache."""
+        Bn, _, Hkv, N, d, bs = self.shape
+        return torch.empty((Bn, Hkv, N // bs, d), dtype=torch.float32, device=self.device)
+
+    def pool_keys(self, k_cache, kp_cache, j_begin: int, j_end: int):
+        """Pool key blocks [j_begin, j_end) of the cache into kp_cache (dsa_pool_keys)."""
+        B.dsa_pool_keys(self.params, k_cache, kp_cache, j_begin, j_end, self.stream)
+        return kp_cache
+
+    def decode(self, q, k_cache, v_cache, kp_cache, length: int, out=None, lse=None, idx=None,
+               cnt=None):
+        """One decode step (dsa_decode_fwd): q [B, Hq, d] at position length - 1."""
+        Bn, Hq, _, _, d, _ = self.shape
+        if out is None:
+            out = torch.empty((Bn, Hq, d), dtype=torch.bfloat16, device=self.device)
+        B.dsa_decode_fwd(self.params, q, k_cache, v_cache, kp_cache, length, out, lse, idx, cnt,
+                         self.ws, self.ws_bytes, self.stream)
+        return out
+
     def check_status(self) -> int:
         return B.dsa_check_status(self.ws, self.stream)

@@ -63,6 +63,9 @@ SIGNATURES = {
     "dsa_select_blocks_static": (ctypes.c_int, [_P, _vp, _vp, _i32p, _i32p, _vp]),
     "dsa_sparse_attn_fwd": (ctypes.c_int, [_P, _vp, _vp, _vp, _i32p, _i32p, _vp, _f32p, _vp, _sz, _vp]),
     "dsa_forward": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _f32p, _i32p, _i32p, _vp, _sz, _vp]),
+    "dsa_pool_keys": (ctypes.c_int, [_P, _vp, _f32p, ctypes.c_int, ctypes.c_int, _vp]),
+    "dsa_decode_fwd": (ctypes.c_int, [_P, _vp, _vp, _vp, _f32p, ctypes.c_int, _vp, _f32p, _i32p, _i32p,
+                                      _vp, _sz, _vp]),
     "dsa_check_status": (ctypes.c_int, [_vp, _vp]),
     "dsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -189,6 +192,18 @@ def dsa_sparse_attn_fwd(p: Params, q, k, v, idx, cnt, out, lse, ws, ws_bytes: in
 def dsa_forward(p: Params, q, k, v, out, lse, idx, cnt, ws, ws_bytes: int, stream=None) -> None:
     _check(_lib.dsa_forward(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(idx),
                             _ptr(cnt), _ptr(ws), ws_bytes, _stream(stream)), "dsa_forward")
+
+
+def dsa_pool_keys(p: Params, k, kp, j_begin: int, j_end: int, stream=None) -> None:
+    _check(_lib.dsa_pool_keys(p.ref, _ptr(k), _ptr(kp), int(j_begin), int(j_end), _stream(stream)),
+           "dsa_pool_keys")
+
+
+def dsa_decode_fwd(p: Params, q, k, v, kp, length: int, out, lse, idx, cnt, ws, ws_bytes: int,
+                   stream=None) -> None:
+    _check(_lib.dsa_decode_fwd(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(kp), int(length), _ptr(out),
+                               _ptr(lse), _ptr(idx), _ptr(cnt), _ptr(ws), ws_bytes, _stream(stream)),
+           "dsa_decode_fwd")
 
 
 def dsa_check_status(ws, stream=None) -> int:

@@ -360,6 +360,41 @@ dsa_status dsa_forward(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k
   return run_attention(p, s, q, k, v, idx, cnt, out, lse, hdr, cs);
 }
 
+dsa_status dsa_pool_keys(const dsa_params* p, const dsa_bf16* k, float* kp, int j_begin, int j_end,
+                         void* stream) {
+  Shape s;
+  dsa_status st = make_shape(p, &s);
+  if (st != DSA_OK) return st;
+  if (is_empty(p)) return DSA_OK;
+  if (j_begin < 0 || j_end < j_begin || j_end > s.nb) return DSA_ERR_INVALID_ARG;
+  if (j_end == j_begin) return DSA_OK;
+  if (k == nullptr || kp == nullptr || !aligned16(k) || !aligned16(kp)) return DSA_ERR_INVALID_ARG;
+  if ((st = check_device()) != DSA_OK) return st;
+  return from_cuda(dsa::launch_pool_range(s, reinterpret_cast<const __nv_bfloat16*>(k), kp, j_begin,
+                                          j_end, (cudaStream_t)stream));
+}
+
+dsa_status dsa_decode_fwd(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k,
+                          const dsa_bf16* v, const float* kp, int length, dsa_bf16* out, float* lse,
+                          int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  dsa_status st = make_shape(p, &s);
+  if (st != DSA_OK) return st;
+  if (is_empty(p)) return DSA_OK;
+  if (length < 1 || length > s.N) return DSA_ERR_INVALID_ARG;
+  if (q == nullptr || k == nullptr || v == nullptr || kp == nullptr || out == nullptr ||
+      !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kp))
+    return DSA_ERR_INVALID_ARG;
+  if ((idx == nullptr) != (cnt == nullptr) && !(idx == nullptr && s.W == 0)) return DSA_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < dsa::kHeaderBytes) return DSA_ERR_WORKSPACE;
+  if ((st = check_device()) != DSA_OK) return st;
+  return from_cuda(dsa::launch_decode(
+      s, budgets(p), reinterpret_cast<const __nv_bfloat16*>(q),
+      reinterpret_cast<const __nv_bfloat16*>(k), reinterpret_cast<const __nv_bfloat16*>(v), kp,
+      length, reinterpret_cast<__nv_bfloat16*>(out), lse, idx, cnt,
+      static_cast<dsa::WsHeader*>(ws), (cudaStream_t)stream));
+}
+
 dsa_status dsa_check_status(void* ws, void* stream) {
   if (ws == nullptr || !aligned16(ws)) return DSA_ERR_WORKSPACE;
   cudaStream_t cs = (cudaStream_t)stream;

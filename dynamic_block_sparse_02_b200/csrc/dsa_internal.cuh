@@ -23,7 +23,8 @@ constexpr int kMaxBlocks = 1024;  // largest nb = N / block
 constexpr int kMaxHeads = 256;    // largest Hq when k_per_head is given
 
 // Kernel ids reported in WsHeader::detail[0].
-enum KernelId { kKernPool = 1, kKernScore = 2, kKernSelect = 3, kKernAttnMma = 4, kKernAttnTc = 5 };
+enum KernelId { kKernPool = 1, kKernScore = 2, kKernSelect = 3, kKernAttnMma = 4, kKernAttnTc = 5,
+                kKernDecode = 6 };
 
 // Derived, validated problem description.
 struct Shape {
@@ -61,6 +62,14 @@ cudaError_t launch_score_select(const Shape& s, const KBudget& kb, const float* 
                                 int32_t* idx, int32_t* cnt, WsHeader* hdr, cudaStream_t st);
 cudaError_t launch_select(const Shape& s, const KBudget& kb, const float* scores, int32_t* idx,
                           int32_t* cnt, WsHeader* hdr, cudaStream_t st);
+// Pooling of key blocks [j0, j1) of every (batch, KV head) of a cache of nb blocks.
+cudaError_t launch_pool_range(const Shape& s, const __nv_bfloat16* k, float* kp, int j0, int j1,
+                              cudaStream_t st);
+// Decode step: one query token per (batch, query head) at position length - 1.
+cudaError_t launch_decode(const Shape& s, const KBudget& kb, const __nv_bfloat16* q,
+                          const __nv_bfloat16* k, const __nv_bfloat16* v, const float* kp,
+                          int length, __nv_bfloat16* out, float* lse, int32_t* idx, int32_t* cnt,
+                          WsHeader* hdr, cudaStream_t st);
 cudaError_t launch_attn_mma(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
                             const __nv_bfloat16* v, const int32_t* idx, const int32_t* cnt,
                             __nv_bfloat16* out, float* lse, WsHeader* hdr, cudaStream_t st);

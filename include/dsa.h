@@ -214,6 +214,34 @@ dsa_status dsa_forward(const dsa_params *p, const dsa_bf16 *q, const dsa_bf16 *k
                        const dsa_bf16 *v, dsa_bf16 *out, float *lse, int32_t *idx,
                        int32_t *cnt, void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * Decode support: pooling of the key cache. kp[b, g, j, :] = mean of key rows
+ * j*block .. j*block+block-1 of k[b, g] (fp32), for j_begin <= j < j_end.
+ * k: bf16 [B, Hkv, N, d] key cache of capacity N = p->N tokens; kp: fp32
+ * [B, Hkv, N/block, d], caller-owned. Call it for each block as it completes.
+ */
+dsa_status dsa_pool_keys(const dsa_params *p, const dsa_bf16 *k, float *kp, int j_begin,
+                         int j_end, void *stream);
+
+/*
+ * Decode step: one new query token per (batch, query head) at position
+ * length - 1 (1 <= length <= N), against the caches k, v bf16 [B, Hkv, N, d]
+ * (rows >= length are not read) and the pooled cache kp (blocks
+ * j < (length-1)/block must be pooled; the token's own block is pooled inside
+ * the call from its present keys). q: bf16 [B, Hq, d]. The token's block row is
+ * selected by p->select_mode exactly as in prefill (scores q . Kp[j]); out:
+ * bf16 [B, Hq, d] = softmax(q K^T * scale) V over the present keys of the kept
+ * blocks; lse: optional fp32 [B, Hq]; idx/cnt: optional int32 [B, Hq, W] /
+ * [B, Hq] (both or neither), the kept blocks. ws: at least the 256-byte header
+ * (dsa_workspace_size is always enough). The zblog.xzdbk.com/559 post (section
+ * 动态开销与计算收益的权衡) keeps the sparse index with the KV cache for
+ * inference; here the pooled keys are kept and the index is re-derived per token.
+ */
+dsa_status dsa_decode_fwd(const dsa_params *p, const dsa_bf16 *q, const dsa_bf16 *k,
+                          const dsa_bf16 *v, const float *kp, int length, dsa_bf16 *out,
+                          float *lse, int32_t *idx, int32_t *cnt, void *ws, size_t ws_bytes,
+                          void *stream);
+
 /* Synchronise `stream`, read the device error flag in the workspace header,
  * clear it, and return it (DSA_OK if no kernel raised one). */
 dsa_status dsa_check_status(void *ws, void *stream);

@@ -388,7 +388,7 @@ def forward(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, block: i
 
 def decode(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, length: int, block: int,
            k_free, local_window: int, n_sink: int, scale: float = 0.0, mode: str = "topk",
-           tau: float = 0.0):
+           tau: float = 0.0, return_scores: bool = False):
     """One decode step: query token q [B, Hq, d] at position length-1, keys and
     values [B, Hkv, >= length, d] (only the first ``length`` are read).
 
@@ -402,7 +402,8 @@ def decode(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, length: i
     reuse it at inference, zblog.xzdbk.com/559 post, section 动态开销与计算收益的
     权衡, point 2).
 
-    Returns idx int32 [B,Hq,W], cnt int32 [B,Hq], out fp64 [B,Hq,d], lse fp64 [B,Hq].
+    Returns idx int32 [B,Hq,W], cnt int32 [B,Hq], out fp64 [B,Hq,d], lse fp64 [B,Hq]
+    (and, with return_scores, the row's block scores [B,Hq,i+1] in fp64).
     """
     q = bf16_to_f64(q_bits)
     k = bf16_to_f64(k_bits)
@@ -449,6 +450,8 @@ def decode(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, length: i
             z = e.sum()
             out[b, h] = (e / z) @ v[b, kv, keys]
             lse[b, h] = mx + math.log(z)
+    if return_scores:
+        return idx, cnt, out, lse, scores
     return idx, cnt, out, lse
 
 

@@ -160,3 +160,24 @@ def test_select_mode_checks():
     ok = B.Params(**base, select_mode=B.DSA_SELECT_GROUP_TOPK)
     assert B.dsa_kmax(ok) == B.dsa_kmax(B.Params(**base))
     assert B.dsa_workspace_size(ok) == B.dsa_workspace_size(B.Params(**base))
+
+
+def test_decode_argument_checks():
+    p = B.Params(B=1, Hq=4, Hkv=2, N=1024, d=64, block=64, k_free=4, local_window=1, n_sink=1)
+    dec = B.raw("dsa_decode_fwd")
+    call = lambda length, q=FAKE, kp=FAKE, out=FAKE, idx=None, cnt=None, ws=FAKE, ws_bytes=256: \
+        dec(p.ref, q, FAKE, FAKE, kp, length, out, None, idx, cnt, ws, ws_bytes, None)
+    assert call(0) == B.DSA_ERR_INVALID_ARG
+    assert call(1025) == B.DSA_ERR_INVALID_ARG
+    assert call(10, q=None) == B.DSA_ERR_INVALID_ARG
+    assert call(10, kp=FAKE + 4) == B.DSA_ERR_INVALID_ARG
+    assert call(10, out=None) == B.DSA_ERR_INVALID_ARG
+    assert call(10, idx=FAKE) == B.DSA_ERR_INVALID_ARG  # idx without cnt
+    assert call(10, ws=None) == B.DSA_ERR_WORKSPACE
+    assert call(10, ws_bytes=255) == B.DSA_ERR_WORKSPACE
+    pool = B.raw("dsa_pool_keys")
+    assert pool(p.ref, FAKE, FAKE, -1, 3, None) == B.DSA_ERR_INVALID_ARG
+    assert pool(p.ref, FAKE, FAKE, 4, 3, None) == B.DSA_ERR_INVALID_ARG
+    assert pool(p.ref, FAKE, FAKE, 0, 17, None) == B.DSA_ERR_INVALID_ARG
+    assert pool(p.ref, FAKE, FAKE, 3, 3, None) == B.DSA_OK  # empty range: nothing to do
+    assert pool(p.ref, None, FAKE, 0, 2, None) == B.DSA_ERR_INVALID_ARG
