@@ -39,6 +39,7 @@ METRIC = "sparse-attn prefill tokens/s at 32K; effective TFLOP/s vs bf16 tensor 
 DEFAULT_WORKLOAD = "32k-gqa"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ATTN_SOURCES = ("attn_tc.cu", "attn_mma.cu")
+SELECT_MODES = {"topk": 0, "group": 1, "threshold": 2}
 
 
 # ---------------------------------------------------------------------------
@@ -300,7 +301,9 @@ def run_ours(args, w):
     q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
     stream = torch.cuda.Stream(device=dev)
     att = BlockSparseAttention.from_workload(w, k_per_head=kph, device=dev, stream=stream,
-                                             attn_kernel=args.attn_kernel)
+                                             attn_kernel=args.attn_kernel,
+                                             select_mode=SELECT_MODES[args.select_mode],
+                                             select_tau=args.tau if args.select_mode == "threshold" else 0.0)
     idx, cnt = att.empty_selection()
     out = att.empty_out()
 
@@ -421,6 +424,113 @@ def run_ours(args, w):
         "clocks": clocks,
         "attn_kernel": {0: "auto", 1: "tcgen05", 2: "mma.sync"}[args.attn_kernel],
     }
+    if args.select_mode != "topk":
+        line["config"]["select_mode"] = args.select_mode
+        if args.select_mode == "threshold":
+            line["config"]["tau"] = args.tau
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# Decode step (one query token per sequence against a full KV cache)
+# ---------------------------------------------------------------------------
+
+DECODE_METRIC = "sparse-attn decode tokens/s at 32K context (one token per sequence per step)"
+
+
+def decode_bytes(w, idx, cnt, length) -> float:
+    """Algorithmic HBM bytes of one decode step: the present keys and values of
+    the union of kept blocks of each KV head's query heads, the pooled key rows
+    of the complete blocks (once per KV head), the query and the output."""
+    total = 0
+    i = (length - 1) // w.block
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            blocks = set()
+            for h in range(g * w.group, (g + 1) * w.group):
+                blocks.update(int(j) for j in idx[b, h, :cnt[b, h]])
+            keys = sum(min((j + 1) * w.block, length) - j * w.block for j in blocks)
+            total += keys * w.d * 2 * 2 + i * w.d * 4
+    total += 2 * w.B * w.Hq * w.d * 2
+    return float(total)
+
+
+def run_decode(args, w):
+    import torch
+    from dynamic_block_sparse_02_b200.attention import BlockSparseAttention
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    length = w.N
+    x = W.make_inputs(w, seed=rank_seed(rank))
+    to_t = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    qtok_h = np.ascontiguousarray(x["q"][:, :, length - 1, :])
+    q = to_t(qtok_h).to(dev)
+    kc, vc = to_t(x["k"]).to(dev), to_t(x["v"]).to(dev)
+    stream = torch.cuda.Stream(device=dev)
+    att = BlockSparseAttention.from_workload(w, device=dev, stream=stream,
+                                             select_mode=SELECT_MODES[args.select_mode],
+                                             select_tau=args.tau if args.select_mode == "threshold" else 0.0)
+    kp = att.pooled_key_cache()
+    idx = torch.empty((w.B, w.Hq, att.width), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.B, w.Hq), dtype=torch.int32, device=dev)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # larger than L2
+    with torch.cuda.stream(stream):
+        att.pool_keys(kc, kp, 0, (length - 1) // w.block)
+        for _ in range(args.warmup):
+            att.decode(q, kc, vc, kp, length, out, None, idx, cnt)
+    torch.cuda.synchronize(dev)
+    from dynamic_block_sparse_02_b200 import binding as B
+    status = B.dsa_check_status(att.ws, stream)
+    if status != B.DSA_OK:
+        raise RuntimeError("device error during warm-up: " + B.status_string(status))
+    ms = []
+    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    if not args.no_clocks:
+        sampler.start()
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            flush.fill_(1)
+            e0.record(stream)
+            att.decode(q, kc, vc, kp, length, out, None, idx, cnt)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms.append(e0.elapsed_time(e1))
+    clocks = sampler.stop()
+    step_ms = statistics.median(ms)
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    nbytes = decode_bytes(w, idx_h, cnt_h, length)
+    peaks, peak_kind = load_peaks()
+    gbs = nbytes / (step_ms / 1e3) / 1e9
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        t0 = time.perf_counter()
+        oracle.decode(qtok_h, x["k"], x["v"], length, w.block, w.k_free, w.local_window, w.n_sink,
+                      mode={"topk": "topk", "group": "group", "threshold": "threshold"}[args.select_mode],
+                      tau=args.tau if args.select_mode == "threshold" else 0.0)
+        spent = time.perf_counter() - t0
+        cpu = {"value": w.B / spent, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"one full decode step ({spent:.2f} s of CPU work)"}
+    cfg = config_dict(w)
+    cfg["l2"] = "L2 flushed (256 MB write) before every timed step"
+    cfg.update({"context": length, "select_mode": args.select_mode})
+    line = {
+        "metric": DECODE_METRIC, "value": w.B / (step_ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                     "frac": gbs / float(peaks["hbm_gbs"]), "traffic": None,
+                     "kernel": "decode (dsa_decode_fwd)", "peak_kind": f"{peak_kind} copy bandwidth",
+                     "algorithmic_bytes": nbytes},
+        "cpu_baseline": cpu,
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
     print(json.dumps(line), flush=True)
     return 0
 
@@ -438,11 +548,18 @@ def main(argv=None):
     ap.add_argument("--ref-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--select-mode", choices=sorted(SELECT_MODES), default="topk",
+                    help="selection rule (default: per-head top-k)")
+    ap.add_argument("--tau", type=float, default=0.05, help="threshold of --select-mode threshold")
+    ap.add_argument("--decode", action="store_true",
+                    help="time one decode step against a full KV cache instead of the prefill step")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.decode:
+        return run_decode(args, w)
     return run_ours(args, w)
 
 
