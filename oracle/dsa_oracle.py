@@ -319,7 +319,8 @@ def sparse_attention(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray,
     """Block-sparse causal attention over the kept blocks, in fp64.
 
     O[b,h,r] = sum over visible kept keys t of softmax_t(q_r . k_t * scale) v_t,
-    with K/V of KV head h // (Hq/Hkv). ``scale`` 0 means 1/sqrt(d).
+    with K/V of KV head h // (Hq/Hkv). ``scale`` 0 means 1/sqrt(d). Inputs are
+    bf16 bit patterns (uint16), widened exactly, or fp64 arrays.
 
     With ``items`` None, returns (O fp64 [B,Hq,N,d], lse fp64 [B,Hq,N]).
     Otherwise ``items`` lists (b, h, i) query blocks and the result is a dict
@@ -345,11 +346,11 @@ def sparse_attention(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray,
         kvh = h // g
         if (b, kvh) not in cache_kv:
             cache_kv.clear()
-            cache_kv[(b, kvh)] = (bf16_to_f64(k_bits[b, kvh]), bf16_to_f64(v_bits[b, kvh]))
+            cache_kv[(b, kvh)] = (_f64(k_bits[b, kvh]), _f64(v_bits[b, kvh]))
         kf, vf = cache_kv[(b, kvh)]
         if (b, h) not in cache_q:
             cache_q.clear()
-            cache_q[(b, h)] = bf16_to_f64(q_bits[b, h])
+            cache_q[(b, h)] = _f64(q_bits[b, h])
         qf = cache_q[(b, h)]
         keys = kept_keys(idx[b, h, i], int(cnt[b, h, i]), block)
         w, l = block_weights(qf[i * block:(i + 1) * block], kf, keys, i, block, scale)
@@ -380,6 +381,96 @@ def forward(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, block: i
     idx, cnt = select_blocks(s, k_free, local_window, n_sink)
     att = sparse_attention(q_bits, k_bits, v_bits, idx, cnt, block, scale, items)
     return idx, cnt, att
+
+
+# ---------------------------------------------------------------------------
+# Backward: gradients of the sparse attention with respect to Q, K and V
+# ---------------------------------------------------------------------------
+
+def _f64(x: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) widened exactly; any other array taken as fp64."""
+    return bf16_to_f64(x) if x.dtype == np.uint16 else np.asarray(x, dtype=np.float64)
+
+
+def sparse_attention_backward(q, k, v, dout, idx: np.ndarray, cnt: np.ndarray, block: int,
+                              scale: float = 0.0,
+                              items: Optional[Iterable[Tuple[int, int, int]]] = None):
+    """Gradients of the block-sparse causal attention, in fp64.
+
+    The pages mention training with the sparse pattern (DeepSeek NSA article,
+    section 2.2) but give no backward rule; the plain reading is the exact
+    gradient of O = softmax(Q K^T * scale) V over the kept, causally visible
+    keys, with the kept lists held fixed (selection is a discrete choice and
+    passes no gradient). Per query block (b, h, i) with kept keys T:
+      P = the softmax weights (block_weights), dP = dO V_T^T,
+      D_r = sum_t P[r, t] dP[r, t]  (equal to dO_r . O_r),
+      dS = P * (dP - D),
+      dQ_i = scale * dS K_T,  dK_T += scale * dS^T Q_i,  dV_T += P^T dO_i,
+    where dK, dV of KV head g sum over its query heads (GQA sharing).
+
+    q, dout: [B, Hq, N, d]; k, v: [B, Hkv, N, d]; bf16 bit patterns (uint16)
+    or fp64. With ``items`` None, returns (dq [B,Hq,N,d], dk [B,Hkv,N,d],
+    dv [B,Hkv,N,d]). Otherwise ``items`` lists (b, h, i) query blocks and the
+    result is (dq_blocks, dk_blocks, dv_blocks): dq_blocks[(b, h, i)] is
+    [block, d]; dk_blocks[(b, g, j)] and dv_blocks[(b, g, j)] are [block, d],
+    the contributions of the listed query blocks to key block j.
+    """
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    g = Hq // Hkv
+    if scale == 0.0:
+        scale = 1.0 / math.sqrt(d)
+    nb = N // block
+    full = items is None
+    if full:
+        items = [(b, h, i) for b in range(B) for h in range(Hq) for i in range(nb)]
+        dq = np.zeros((B, Hq, N, d))
+        dk = np.zeros((B, Hkv, N, d))
+        dv = np.zeros((B, Hkv, N, d))
+    else:
+        dq_b, dk_b, dv_b = {}, {}, {}
+    items = sorted(items)
+    cache_kv, cache_q = {}, {}
+    for (b, h, i) in items:
+        kvh = h // g
+        if (b, kvh) not in cache_kv:
+            cache_kv.clear()
+            cache_kv[(b, kvh)] = (_f64(k[b, kvh]), _f64(v[b, kvh]))
+        kf, vf = cache_kv[(b, kvh)]
+        if (b, h) not in cache_q:
+            cache_q.clear()
+            cache_q[(b, h)] = (_f64(q[b, h]), _f64(dout[b, h]))
+        qf, dof = cache_q[(b, h)]
+        rows = slice(i * block, (i + 1) * block)
+        keys = kept_keys(idx[b, h, i], int(cnt[b, h, i]), block)
+        if keys.size == 0:
+            if not full:
+                dq_b[(b, h, i)] = np.zeros((block, d))
+            continue
+        qb, dob = qf[rows], dof[rows]
+        w, _ = block_weights(qb, kf, keys, i, block, scale)
+        kt, vt = kf[keys], vf[keys]
+        dp = dob @ vt.T
+        drow = (w * dp).sum(axis=1)
+        ds = w * (dp - drow[:, None])
+        dq_i = scale * (ds @ kt)
+        dk_t = scale * (ds.T @ qb)
+        dv_t = w.T @ dob
+        if full:
+            dq[b, h, rows] = dq_i
+            np.add.at(dk[b, kvh], keys, dk_t)
+            np.add.at(dv[b, kvh], keys, dv_t)
+        else:
+            dq_b[(b, h, i)] = dq_i
+            for c, j in enumerate(np.asarray(idx[b, h, i][:int(cnt[b, h, i])], dtype=np.int64)):
+                sl = slice(c * block, (c + 1) * block)
+                key = (b, kvh, int(j))
+                if key not in dk_b:
+                    dk_b[key] = np.zeros((block, d))
+                    dv_b[key] = np.zeros((block, d))
+                dk_b[key] += dk_t[sl]
+                dv_b[key] += dv_t[sl]
+    return (dq, dk, dv) if full else (dq_b, dk_b, dv_b)
 
 
 # ---------------------------------------------------------------------------

@@ -560,3 +560,124 @@ def test_decode_group_of_identical_heads_equals_per_head():
     b = oracle.decode(q, k, v, L, bs, 4, 2, 1, mode="group")
     for x, y in zip(a, b):
         np.testing.assert_array_equal(x, y)
+
+
+# ---------------------------------------------------------------------------
+# Backward (gradients of the sparse attention)
+# ---------------------------------------------------------------------------
+
+def _mixed_lists(B, Hq, nb, seed, keep_prob=0.6):
+    """Random kept lists: the diagonal always, other causal blocks at random."""
+    g = np.random.default_rng(seed)
+    idx = np.full((B, Hq, nb, nb), -1, dtype=np.int32)
+    cnt = np.zeros((B, Hq, nb), dtype=np.int32)
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(nb):
+                lst = [j for j in range(i) if g.random() < keep_prob] + [i]
+                idx[b, h, i, :len(lst)] = lst
+                cnt[b, h, i] = len(lst)
+    return idx, cnt
+
+
+def _loss(q, k, v, gout, idx, cnt, bs):
+    o, _ = oracle.sparse_attention(q, k, v, idx, cnt, bs)
+    return float((o * gout).sum())
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_backward_matches_central_differences(seed):
+    # L = sum(O * G) has dL/dO = G, so the gradients must equal the central
+    # differences of the oracle's own forward along random directions
+    B, Hq, Hkv, N, d, bs = 1, 4, 2, 12, 4, 3
+    g = np.random.default_rng(100 + seed)
+    q = g.standard_normal((B, Hq, N, d))
+    k = g.standard_normal((B, Hkv, N, d))
+    v = g.standard_normal((B, Hkv, N, d))
+    gout = g.standard_normal((B, Hq, N, d))
+    idx, cnt = _mixed_lists(B, Hq, N // bs, seed)
+    dq, dk, dv = oracle.sparse_attention_backward(q, k, v, gout, idx, cnt, bs)
+    eps = 1e-6
+    for name, x, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for t in range(3):
+            u = g.standard_normal(x.shape)
+            args = {"q": q, "k": k, "v": v}
+            args[name] = x + eps * u
+            lp = _loss(args["q"], args["k"], args["v"], gout, idx, cnt, bs)
+            args[name] = x - eps * u
+            lm = _loss(args["q"], args["k"], args["v"], gout, idx, cnt, bs)
+            fd = (lp - lm) / (2 * eps)
+            an = float((grad * u).sum())
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+def test_backward_dense_lists_match_autograd_of_causal_attention():
+    # every causal block kept: the gradients are those of dense causal
+    # attention, here through PyTorch's autograd on the textbook routine
+    B, Hq, Hkv, N, d, bs = 1, 4, 2, 16, 8, 4
+    q = rand_bits((B, Hq, N, d), 11)
+    k = rand_bits((B, Hkv, N, d), 12)
+    v = rand_bits((B, Hkv, N, d), 13)
+    do = rand_bits((B, Hq, N, d), 14)
+    nb = N // bs
+    idx = np.full((B, Hq, nb, nb), -1, dtype=np.int32)
+    cnt = np.zeros((B, Hq, nb), dtype=np.int32)
+    for i in range(nb):
+        idx[:, :, i, :i + 1] = np.arange(i + 1)
+        cnt[:, :, i] = i + 1
+    dq, dk, dv = oracle.sparse_attention_backward(q, k, v, do, idx, cnt, bs)
+    qt, kt, vt = (f64(x).requires_grad_(True) for x in (q, k, v))
+    o = F.scaled_dot_product_attention(qt, kt.repeat_interleave(Hq // Hkv, 1),
+                                       vt.repeat_interleave(Hq // Hkv, 1), is_causal=True)
+    o.backward(f64(do))
+    np.testing.assert_allclose(dq, qt.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk, kt.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv, vt.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_backward_invariants():
+    B, Hq, Hkv, N, d, bs = 2, 4, 2, 24, 8, 4
+    q = rand_bits((B, Hq, N, d), 21)
+    k = rand_bits((B, Hkv, N, d), 22)
+    v = rand_bits((B, Hkv, N, d), 23)
+    do = rand_bits((B, Hq, N, d), 24)
+    idx, cnt = _mixed_lists(B, Hq, N // bs, 25, keep_prob=0.4)
+    dq, dk, dv = oracle.sparse_attention_backward(q, k, v, do, idx, cnt, bs)
+    g = Hq // Hkv
+    # softmax weights sum to one: sum over keys of dV is the sum of dO over the
+    # group's query rows (every row sees at least its own key)
+    dof = oracle.bf16_to_f64(do)
+    for b in range(B):
+        for kvh in range(Hkv):
+            np.testing.assert_allclose(dv[b, kvh].sum(axis=0), dof[b, kvh * g:(kvh + 1) * g].sum(axis=(0, 1)),
+                                       rtol=1e-10, atol=1e-10)
+            # shifting every key by one vector shifts each row's logits by a
+            # constant: the softmax, hence the loss, does not move
+            np.testing.assert_allclose(dk[b, kvh].sum(axis=0), 0.0, atol=1e-10)
+    # query row 0 sees only key 0: its softmax is constant, its gradient 0
+    np.testing.assert_allclose(dq[:, :, 0], 0.0, atol=1e-14)
+    # a key block that no list keeps receives no gradient
+    kept = np.zeros((B, Hkv, N // bs), dtype=bool)
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(N // bs):
+                kept[b, h // g, idx[b, h, i, :cnt[b, h, i]]] = True
+    for b, kvh, j in zip(*np.nonzero(~kept)):
+        assert np.all(dk[b, kvh, j * bs:(j + 1) * bs] == 0) and np.all(dv[b, kvh, j * bs:(j + 1) * bs] == 0)
+
+
+def test_backward_items_equal_the_full_result():
+    B, Hq, Hkv, N, d, bs = 1, 4, 1, 16, 8, 4
+    q = rand_bits((B, Hq, N, d), 31)
+    k = rand_bits((B, Hkv, N, d), 32)
+    v = rand_bits((B, Hkv, N, d), 33)
+    do = rand_bits((B, Hq, N, d), 34)
+    idx, cnt = _mixed_lists(B, Hq, N // bs, 35)
+    dq, dk, dv = oracle.sparse_attention_backward(q, k, v, do, idx, cnt, bs)
+    # dK/dV of key block 1: the query blocks whose lists keep it
+    items = [(0, h, i) for h in range(Hq) for i in range(N // bs) if 1 in idx[0, h, i, :cnt[0, h, i]]]
+    items = sorted(set(items) | {(0, 2, 3)})
+    dqb, dkb, dvb = oracle.sparse_attention_backward(q, k, v, do, idx, cnt, bs, items=items)
+    np.testing.assert_allclose(dqb[(0, 2, 3)], dq[0, 2, 12:16], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dkb[(0, 0, 1)], dk[0, 0, 4:8], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dvb[(0, 0, 1)], dv[0, 0, 4:8], rtol=0, atol=1e-13)
