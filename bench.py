@@ -478,6 +478,7 @@ def run_decode(args, w):
     cnt = torch.empty((w.B, w.Hq), dtype=torch.int32, device=dev)
     out = torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # larger than L2
+    clean = torch.ones(256 << 20, dtype=torch.uint8, device=dev)   # read after the flush
     with torch.cuda.stream(stream):
         att.pool_keys(kc, kp, 0, (length - 1) // w.block)
         for _ in range(args.warmup):
@@ -487,21 +488,30 @@ def run_decode(args, w):
     status = B.dsa_check_status(att.ws, stream)
     if status != B.DSA_OK:
         raise RuntimeError("device error during warm-up: " + B.status_string(status))
-    ms = []
+    # Each timed step starts from a cold L2: a 256 MB write (the flush), then a
+    # 256 MB read, which evicts the flush's dirty lines so that the step's reads
+    # do not pay for their write-back. The write-only flush is timed too.
+    def timed(read_after):
+        ms = []
+        for _ in range(args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                flush.fill_(1)
+                if read_after:
+                    clean.max()
+                e0.record(stream)
+                att.decode(q, kc, vc, kp, length, out, None, idx, cnt)
+                e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ms.append(e0.elapsed_time(e1))
+        return statistics.median(ms)
+
     sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
     if not args.no_clocks:
         sampler.start()
-    for _ in range(args.steps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            flush.fill_(1)
-            e0.record(stream)
-            att.decode(q, kc, vc, kp, length, out, None, idx, cnt)
-            e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms.append(e0.elapsed_time(e1))
+    step_ms = timed(True)
     clocks = sampler.stop()
-    step_ms = statistics.median(ms)
+    dirty_ms = timed(False)
     idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
     nbytes = decode_bytes(w, idx_h, cnt_h, length)
     peaks, peak_kind = load_peaks()
@@ -517,7 +527,8 @@ def run_decode(args, w):
         cpu = {"value": w.B / spent, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                "sample": f"one full decode step ({spent:.2f} s of CPU work)"}
     cfg = config_dict(w)
-    cfg["l2"] = "L2 flushed (256 MB write) before every timed step"
+    cfg["l2"] = ("L2 flushed before every timed step: 256 MB write, then 256 MB read "
+                 "(clean cold L2); ms_per_step_dirty_l2 = the same after the write alone")
     cfg.update({"context": length, "select_mode": args.select_mode})
     line = {
         "metric": DECODE_METRIC, "value": w.B / (step_ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
@@ -528,7 +539,94 @@ def run_decode(args, w):
                      "kernel": "decode (dsa_decode_fwd)", "peak_kind": f"{peak_kind} copy bandwidth",
                      "algorithmic_bytes": nbytes},
         "cpu_baseline": cpu,
-        "gpu_launches": args.steps,
+        "ms_per_step_dirty_l2": dirty_ms,
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+BACKWARD_METRIC = "sparse-attn backward tokens/s at 32K (dQ, dK, dV over the kept blocks)"
+
+
+def backward_flops(cnt_sum: int, block: int, d: int) -> float:
+    """Algorithmic FLOPs of the backward: 10 * bs^2 * d per kept block (the five
+    products S = Q K^T, dP = dO V^T, dV = P^T dO, dK = dS^T Q, dQ = dS K over
+    full tiles). The kernels recompute S and dP in both the dQ and the dK/dV
+    pass; that recomputation is not counted."""
+    return 10.0 * block * block * d * cnt_sum
+
+
+def run_backward(args, w):
+    import torch
+    from dynamic_block_sparse_02_b200 import binding as B
+    from dynamic_block_sparse_02_b200.attention import BlockSparseAttention
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    x = W.make_inputs(w, seed=rank_seed(rank))
+    g = np.random.default_rng(1000 + rank)
+    do_h = W.f32_to_bf16_bits(g.standard_normal(x["q"].shape).astype(np.float32))
+    to_t = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    q, k, v, dout = (to_t(a).to(dev) for a in (x["q"], x["k"], x["v"], do_h))
+    stream = torch.cuda.Stream(device=dev)
+    att = BlockSparseAttention.from_workload(w, device=dev, stream=stream)
+    idx, cnt = att.empty_selection()
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    with torch.cuda.stream(stream):
+        att.forward(q, k, v, out, lse, idx, cnt)  # the selection and forward the backward follows
+        for _ in range(args.warmup):
+            att.sparse_attn_backward(q, k, v, out, lse, dout, idx, cnt, dq, dk, dv)
+    torch.cuda.synchronize(dev)
+    status = B.dsa_check_status(att.ws, stream)
+    if status != B.DSA_OK:
+        raise RuntimeError("device error during warm-up: " + B.status_string(status))
+    kept = int(cnt.sum().item())
+    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    if not args.no_clocks:
+        sampler.start()
+    ms = []
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            att.sparse_attn_backward(q, k, v, out, lse, dout, idx, cnt, dq, dk, dv)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms.append(e0.elapsed_time(e1))
+    clocks = sampler.stop()
+    step_ms = statistics.median(ms)
+    peaks, peak_kind = load_peaks()
+    flops = backward_flops(kept, w.block, w.d)
+    tfs = flops / (step_ms / 1e3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+        items = [(0, h, i) for h in range(w.Hq) for i in range(w.nb - 1, -1, -97)][:args.bwd_sample]
+        t0 = time.perf_counter()
+        oracle.sparse_attention_backward(x["q"], x["k"], x["v"], do_h, idx_h, cnt_h, w.block, items=items)
+        spent = time.perf_counter() - t0
+        cpu = {"value": len(items) * w.block / spent, "unit": "tokens/s", "cores": blas_threads(),
+               "kind": "oracle", "sample": f"{len(items)} query blocks of the workload ({spent:.1f} s)"}
+    cfg = config_dict(w)
+    cfg["l2"] = "inputs larger than L2 (q, dout, out 268 MB each), no flush"
+    cfg["selection"] = "the forward's own top-k lists"
+    line = {
+        "metric": BACKWARD_METRIC, "value": w.B * w.N / (step_ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+        "roofline": {"bound": "tensor", "achieved": tfs, "peak": peak, "unit": "TFLOP/s", "frac": tfs / peak,
+                     "traffic": None, "kernel": "backward step (prep, colbits, dq, dkv)",
+                     "peak_kind": f"{peak_kind} sustained bf16", "algorithmic_flops": flops},
+        "kept_blocks": kept,
+        "cpu_baseline": cpu,
+        "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
@@ -553,6 +651,9 @@ def main(argv=None):
     ap.add_argument("--tau", type=float, default=0.05, help="threshold of --select-mode threshold")
     ap.add_argument("--decode", action="store_true",
                     help="time one decode step against a full KV cache instead of the prefill step")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward over the kept blocks instead of the prefill step")
+    ap.add_argument("--bwd-sample", type=int, default=1024, help="query blocks in the oracle's timed sample")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     w = WORKLOADS[args.workload]
@@ -560,6 +661,8 @@ def main(argv=None):
         return run_reference(args, w)
     if args.decode:
         return run_decode(args, w)
+    if args.backward:
+        return run_backward(args, w)
     return run_ours(args, w)
 
 

@@ -95,6 +95,16 @@ class BlockSparseAttention:
                               self.stream)
         return out
 
+    def sparse_attn_backward(self, q, k, v, out, lse, dout, idx, cnt, dq=None, dk=None, dv=None):
+        """Gradients of sparse_attn over the kept blocks (dsa_sparse_attn_bwd); out and
+        lse are the forward's outputs for the same idx/cnt. Returns (dq, dk, dv)."""
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(k) if dk is None else dk
+        dv = torch.empty_like(v) if dv is None else dv
+        B.dsa_sparse_attn_bwd(self.params, q, k, v, out, lse, dout, idx, cnt, dq, dk, dv, self.ws,
+                              self.ws_bytes, self.stream)
+        return dq, dk, dv
+
     def pooled_key_cache(self):
         """An fp32 [B, Hkv, N/block, d] buffer for the pooled key cache."""
         Bn, _, Hkv, N, d, bs = self.shape

@@ -62,6 +62,8 @@ SIGNATURES = {
     "dsa_select_blocks": (ctypes.c_int, [_P, _vp, _vp, _i32p, _i32p, _vp, _sz, _vp]),
     "dsa_select_blocks_static": (ctypes.c_int, [_P, _vp, _vp, _i32p, _i32p, _vp]),
     "dsa_sparse_attn_fwd": (ctypes.c_int, [_P, _vp, _vp, _vp, _i32p, _i32p, _vp, _f32p, _vp, _sz, _vp]),
+    "dsa_sparse_attn_bwd": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _f32p, _vp, _i32p, _i32p, _vp, _vp,
+                                           _vp, _vp, _sz, _vp]),
     "dsa_forward": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _f32p, _i32p, _i32p, _vp, _sz, _vp]),
     "dsa_pool_keys": (ctypes.c_int, [_P, _vp, _f32p, ctypes.c_int, ctypes.c_int, _vp]),
     "dsa_decode_fwd": (ctypes.c_int, [_P, _vp, _vp, _vp, _f32p, ctypes.c_int, _vp, _f32p, _i32p, _i32p,
@@ -187,6 +189,14 @@ def dsa_sparse_attn_fwd(p: Params, q, k, v, idx, cnt, out, lse, ws, ws_bytes: in
     _check(_lib.dsa_sparse_attn_fwd(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt),
                                     _ptr(out), _ptr(lse), _ptr(ws), ws_bytes, _stream(stream)),
            "dsa_sparse_attn_fwd")
+
+
+def dsa_sparse_attn_bwd(p: Params, q, k, v, out, lse, dout, idx, cnt, dq, dk, dv, ws, ws_bytes: int,
+                        stream=None) -> None:
+    _check(_lib.dsa_sparse_attn_bwd(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout),
+                                    _ptr(idx), _ptr(cnt), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                                    ws_bytes, _stream(stream)),
+           "dsa_sparse_attn_bwd")
 
 
 def dsa_forward(p: Params, q, k, v, out, lse, idx, cnt, ws, ws_bytes: int, stream=None) -> None:

@@ -233,7 +233,13 @@ dsa_status dsa_workspace_size(const dsa_params* p, size_t* bytes) {
   Shape s;
   dsa_status st = make_shape(p, &s);
   if (st != DSA_OK) return st;
-  *bytes = is_empty(p) ? dsa::kHeaderBytes : layout(s).total;
+  if (is_empty(p)) {
+    *bytes = dsa::kHeaderBytes;
+  } else {
+    const size_t a = layout(s).total, b = dsa::decode_ws_layout(s).total;
+    const size_t c = dsa::bwd_ws_layout(s).total;
+    *bytes = a > b ? (a > c ? a : c) : (b > c ? b : c);
+  }
   return DSA_OK;
 }
 
@@ -333,6 +339,30 @@ dsa_status dsa_sparse_attn_fwd(const dsa_params* p, const dsa_bf16* q, const dsa
   return run_attention(p, s, q, k, v, idx, cnt, out, lse, hdr, (cudaStream_t)stream);
 }
 
+dsa_status dsa_sparse_attn_bwd(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k,
+                               const dsa_bf16* v, const dsa_bf16* out, const float* lse,
+                               const dsa_bf16* dout, const int32_t* idx, const int32_t* cnt,
+                               dsa_bf16* dq, dsa_bf16* dk, dsa_bf16* dv, void* ws, size_t ws_bytes,
+                               void* stream) {
+  Shape s;
+  dsa_status st = make_shape(p, &s);
+  if (st != DSA_OK) return st;
+  if (is_empty(p)) return DSA_OK;
+  const void* need16[] = {q, k, v, out, dout, dq, dk, dv};
+  for (const void* ptr : need16)
+    if (ptr == nullptr || !aligned16(ptr)) return DSA_ERR_INVALID_ARG;
+  if (lse == nullptr || !aligned16(lse) || cnt == nullptr || (idx == nullptr && s.W > 0))
+    return DSA_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < dsa::bwd_ws_layout(s).total) return DSA_ERR_WORKSPACE;
+  if ((st = check_device()) != DSA_OK) return st;
+  return from_cuda(dsa::launch_attn_bwd(
+      s, reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k),
+      reinterpret_cast<const __nv_bfloat16*>(v), reinterpret_cast<const __nv_bfloat16*>(out), lse,
+      reinterpret_cast<const __nv_bfloat16*>(dout), idx, cnt, reinterpret_cast<__nv_bfloat16*>(dq),
+      reinterpret_cast<__nv_bfloat16*>(dk), reinterpret_cast<__nv_bfloat16*>(dv), ws,
+      (cudaStream_t)stream));
+}
+
 dsa_status dsa_forward(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k, const dsa_bf16* v,
                        dsa_bf16* out, float* lse, int32_t* idx, int32_t* cnt, void* ws,
                        size_t ws_bytes, void* stream) {
@@ -386,13 +416,14 @@ dsa_status dsa_decode_fwd(const dsa_params* p, const dsa_bf16* q, const dsa_bf16
       !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kp))
     return DSA_ERR_INVALID_ARG;
   if ((idx == nullptr) != (cnt == nullptr) && !(idx == nullptr && s.W == 0)) return DSA_ERR_INVALID_ARG;
-  if (ws == nullptr || !aligned16(ws) || ws_bytes < dsa::kHeaderBytes) return DSA_ERR_WORKSPACE;
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < dsa::decode_ws_layout(s).total)
+    return DSA_ERR_WORKSPACE;
   if ((st = check_device()) != DSA_OK) return st;
   return from_cuda(dsa::launch_decode(
       s, budgets(p), reinterpret_cast<const __nv_bfloat16*>(q),
       reinterpret_cast<const __nv_bfloat16*>(k), reinterpret_cast<const __nv_bfloat16*>(v), kp,
       length, reinterpret_cast<__nv_bfloat16*>(out), lse, idx, cnt,
-      static_cast<dsa::WsHeader*>(ws), (cudaStream_t)stream));
+      ws, (cudaStream_t)stream));
 }
 
 dsa_status dsa_check_status(void* ws, void* stream) {

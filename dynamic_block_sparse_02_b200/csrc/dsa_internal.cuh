@@ -24,7 +24,7 @@ constexpr int kMaxHeads = 256;    // largest Hq when k_per_head is given
 
 // Kernel ids reported in WsHeader::detail[0].
 enum KernelId { kKernPool = 1, kKernScore = 2, kKernSelect = 3, kKernAttnMma = 4, kKernAttnTc = 5,
-                kKernDecode = 6 };
+                kKernDecode = 6, kKernAttnBwd = 7 };
 
 // Derived, validated problem description.
 struct Shape {
@@ -65,11 +65,66 @@ cudaError_t launch_select(const Shape& s, const KBudget& kb, const float* scores
 // Pooling of key blocks [j0, j1) of every (batch, KV head) of a cache of nb blocks.
 cudaError_t launch_pool_range(const Shape& s, const __nv_bfloat16* k, float* kp, int j0, int j1,
                               cudaStream_t st);
+// Decode workspace after the header: fp32 scores [B, Hq, nb] (per-head rows;
+// the group-shared rule uses the first B*Hkv rows for the groups' sums), fp32
+// partial softmax states [B, Hq, kDecMaxSplit', d + 4] (output row, m, l) with
+// kDecMaxSplit' = min(kDecMaxSplit, nb) splits of a head's kept blocks, and one
+// arrival counter per (batch, KV head, chunk of 8 query heads).
+constexpr int kDecMaxSplit = 64;
+constexpr int kDecHeadChunk = 8;
+struct DecodeWs {
+  size_t scores, part, ctr, total;
+  int smax;
+};
+inline size_t ws_round_up(size_t x) { return (x + 255) / 256 * 256; }
+inline DecodeWs decode_ws_layout(const Shape& s) {
+  DecodeWs w;
+  w.smax = s.nb < kDecMaxSplit ? s.nb : kDecMaxSplit;
+  const int hc = (s.group + kDecHeadChunk - 1) / kDecHeadChunk;
+  size_t off = kHeaderBytes;
+  w.scores = off;
+  off += ws_round_up((size_t)s.B * s.Hq * s.nb * sizeof(float));
+  w.part = off;
+  off += ws_round_up((size_t)s.B * s.Hq * w.smax * (s.d + 4) * sizeof(float));
+  w.ctr = off;
+  off += ws_round_up((size_t)s.B * s.Hkv * hc * sizeof(int));
+  w.total = off;
+  return w;
+}
+
+// Backward workspace after the header: fp32 D_r = dO_r . O_r and base-2 lse
+// per query row [B, Hq, N], and the transposed kept lists, one bitmap of
+// cw = ceil(G * nb / 32) words per key block [B, Hkv, nb, cw].
+struct BwdWs {
+  size_t drow, lse2, colbits, total;
+  int cw;
+};
+inline BwdWs bwd_ws_layout(const Shape& s) {
+  BwdWs w;
+  w.cw = (s.group * s.nb + 31) / 32;
+  size_t off = kHeaderBytes;
+  w.drow = off;
+  off += ws_round_up((size_t)s.B * s.Hq * s.N * sizeof(float));
+  w.lse2 = off;
+  off += ws_round_up((size_t)s.B * s.Hq * s.N * sizeof(float));
+  w.colbits = off;
+  off += ws_round_up((size_t)s.B * s.Hkv * s.nb * w.cw * sizeof(uint32_t));
+  w.total = off;
+  return w;
+}
+
+// Backward of the sparse attention over the kept blocks (dQ, dK, dV).
+cudaError_t launch_attn_bwd(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                            const __nv_bfloat16* v, const __nv_bfloat16* o, const float* lse,
+                            const __nv_bfloat16* dout, const int32_t* idx, const int32_t* cnt,
+                            __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, void* ws,
+                            cudaStream_t st);
+
 // Decode step: one query token per (batch, query head) at position length - 1.
 cudaError_t launch_decode(const Shape& s, const KBudget& kb, const __nv_bfloat16* q,
                           const __nv_bfloat16* k, const __nv_bfloat16* v, const float* kp,
                           int length, __nv_bfloat16* out, float* lse, int32_t* idx, int32_t* cnt,
-                          WsHeader* hdr, cudaStream_t st);
+                          void* ws, cudaStream_t st);
 cudaError_t launch_attn_mma(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
                             const __nv_bfloat16* v, const int32_t* idx, const int32_t* cnt,
                             __nv_bfloat16* out, float* lse, WsHeader* hdr, cudaStream_t st);

@@ -207,6 +207,30 @@ dsa_status dsa_sparse_attn_fwd(const dsa_params *p, const dsa_bf16 *q, const dsa
                                void *stream);
 
 /*
+ * Backward of step 4: gradients of the attention over the kept blocks with
+ * the kept lists held fixed (the selection is a discrete choice and passes no
+ * gradient). The DeepSeek NSA article (section 2.2) trains with the sparse
+ * pattern but states no backward rule; this is the exact gradient of
+ * O = softmax(Q K^T * scale) V over the kept, causally visible keys:
+ * P = exp(S * scale - lse), dP = dO V^T, D = rowsum(dO * O),
+ * dS = P * (dP - D), dQ = scale * dS K, dK = scale * dS^T Q, dV = P^T dO,
+ * with dK, dV of a KV head summed over its query heads.
+ * q, out, dout, dq: bf16 [B, Hq, N, d]; k, v, dk, dv: bf16 [B, Hkv, N, d];
+ * out and lse (fp32 [B, Hq, N], natural log, -inf for a row with no visible
+ * key) are the forward's outputs for the same idx/cnt (int32 [B, Hq, nb, W]
+ * and [B, Hq, nb]). dq, dk, dv are written in full (zero where nothing
+ * contributes); all pointers 16-byte aligned and device-resident. ws: at
+ * least dsa_workspace_size bytes. Entries outside 0 <= j <= i are skipped and
+ * raise DSA_ERR_DEVICE_BOUNDS. The sums run in a fixed order: the results are
+ * deterministic.
+ */
+dsa_status dsa_sparse_attn_bwd(const dsa_params *p, const dsa_bf16 *q, const dsa_bf16 *k,
+                               const dsa_bf16 *v, const dsa_bf16 *out, const float *lse,
+                               const dsa_bf16 *dout, const int32_t *idx, const int32_t *cnt,
+                               dsa_bf16 *dq, dsa_bf16 *dk, dsa_bf16 *dv, void *ws,
+                               size_t ws_bytes, void *stream);
+
+/*
  * Steps 1-4 in one call; the scores never reach device memory. idx/cnt are
  * optional outputs (NULL keeps them in the workspace); lse is optional.
  */
@@ -232,8 +256,8 @@ dsa_status dsa_pool_keys(const dsa_params *p, const dsa_bf16 *k, float *kp, int 
  * selected by p->select_mode exactly as in prefill (scores q . Kp[j]); out:
  * bf16 [B, Hq, d] = softmax(q K^T * scale) V over the present keys of the kept
  * blocks; lse: optional fp32 [B, Hq]; idx/cnt: optional int32 [B, Hq, W] /
- * [B, Hq] (both or neither), the kept blocks. ws: at least the 256-byte header
- * (dsa_workspace_size is always enough). The zblog.xzdbk.com/559 post (section
+ * [B, Hq] (both or neither), the kept blocks. ws: at least dsa_workspace_size
+ * bytes (scores, partial softmax states of the splits, arrival counters). The zblog.xzdbk.com/559 post (section
  * 动态开销与计算收益的权衡) keeps the sparse index with the KV cache for
  * inference; here the pooled keys are kept and the index is re-derived per token.
  */

@@ -26,6 +26,7 @@ def declared_functions():
 def test_header_declares_expected_entry_points():
     names = declared_functions()
     for n in ("dsa_block_scores", "dsa_topk_select", "dsa_sparse_attn_fwd", "dsa_forward",
+              "dsa_sparse_attn_bwd", "dsa_decode_fwd", "dsa_pool_keys",
               "dsa_workspace_size", "dsa_kmax", "dsa_check_status", "dsa_status_string"):
         assert n in names
 
@@ -62,9 +63,14 @@ def test_kmax_and_workspace_size(name):
     assert width == expect
     ws = B.dsa_workspace_size(p)
     rnd = lambda x: (x + 255) // 256 * 256
-    expect_ws = 256 + rnd(w.B * w.Hq * w.nb * w.d * 4) + rnd(w.B * w.Hkv * w.nb * w.d * 4) \
+    prefill = 256 + rnd(w.B * w.Hq * w.nb * w.d * 4) + rnd(w.B * w.Hkv * w.nb * w.d * 4) \
         + rnd(w.B * w.Hq * w.nb * width * 4) + rnd(w.B * w.Hq * w.nb * 4)
-    assert ws == expect_ws
+    # decode: scores [B, Hq, nb], partial states [B, Hq, min(64, nb), d + 4], counters
+    decode = 256 + rnd(w.B * w.Hq * w.nb * 4) + rnd(w.B * w.Hq * min(64, w.nb) * (w.d + 4) * 4) \
+        + rnd(w.B * w.Hkv * -(-(w.Hq // w.Hkv) // 8) * 4)
+    # backward: D and base-2 lse per query row, one bitmap of ceil(G * nb / 32) words per key block
+    backward = 256 + 2 * rnd(w.B * w.Hq * w.N * 4) + rnd(w.B * w.Hkv * w.nb * -(-(w.Hq // w.Hkv * w.nb) // 32) * 4)
+    assert ws == max(prefill, decode, backward)
 
 
 def status_of_forward(p, q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=None, idx=None, cnt=None, ws=FAKE,
@@ -124,7 +130,13 @@ def test_null_and_misaligned_pointers_rejected():
 
 def test_workspace_checks():
     p = B.Params(**BASE)
-    need = B.dsa_workspace_size(p)
+    # the forward's own part: header, pooled Q and K, idx and cnt rows
+    b, hq, hkv, n, d, bs = (BASE[x] for x in ("B", "Hq", "Hkv", "N", "d", "block"))
+    nb, width = n // bs, B.dsa_kmax(p)
+    rnd = lambda x: (x + 255) // 256 * 256
+    need = 256 + rnd(b * hq * nb * d * 4) + rnd(b * hkv * nb * d * 4) + rnd(b * hq * nb * width * 4) \
+        + rnd(b * hq * nb * 4)
+    assert need <= B.dsa_workspace_size(p)
     assert status_of_forward(p, ws=None) == B.DSA_ERR_WORKSPACE
     assert status_of_forward(p, ws_bytes=need - 1) == B.DSA_ERR_WORKSPACE
     assert status_of_forward(p, ws=FAKE + 8) == B.DSA_ERR_WORKSPACE
@@ -175,9 +187,34 @@ def test_decode_argument_checks():
     assert call(10, idx=FAKE) == B.DSA_ERR_INVALID_ARG  # idx without cnt
     assert call(10, ws=None) == B.DSA_ERR_WORKSPACE
     assert call(10, ws_bytes=255) == B.DSA_ERR_WORKSPACE
+    # the decode's own workspace: header, scores [1, 4, 16], partial states [1, 4, 16, 68], counters
+    need = 256 + 256 + 4 * 16 * 68 * 4 + 256
+    assert need <= B.dsa_workspace_size(p)
+    assert call(10, ws_bytes=need - 1) == B.DSA_ERR_WORKSPACE
     pool = B.raw("dsa_pool_keys")
     assert pool(p.ref, FAKE, FAKE, -1, 3, None) == B.DSA_ERR_INVALID_ARG
     assert pool(p.ref, FAKE, FAKE, 4, 3, None) == B.DSA_ERR_INVALID_ARG
     assert pool(p.ref, FAKE, FAKE, 0, 17, None) == B.DSA_ERR_INVALID_ARG
     assert pool(p.ref, FAKE, FAKE, 3, 3, None) == B.DSA_OK  # empty range: nothing to do
     assert pool(p.ref, None, FAKE, 0, 2, None) == B.DSA_ERR_INVALID_ARG
+
+
+def test_backward_argument_checks():
+    p = B.Params(B=1, Hq=4, Hkv=2, N=1024, d=64, block=64, k_free=4, local_window=1, n_sink=1)
+    bwd = B.raw("dsa_sparse_attn_bwd")
+
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, dout=FAKE, idx=FAKE, cnt=FAKE, dq=FAKE,
+                 dk=FAKE, dv=FAKE, ws=FAKE, ws_bytes=1 << 40)
+        a.update(kw)
+        return bwd(p.ref, a["q"], a["k"], a["v"], a["out"], a["lse"], a["dout"], a["idx"], a["cnt"],
+                   a["dq"], a["dk"], a["dv"], a["ws"], a["ws_bytes"], None)
+
+    for name in ("q", "k", "v", "out", "lse", "dout", "idx", "cnt", "dq", "dk", "dv"):
+        assert call(**{name: None}) == B.DSA_ERR_INVALID_ARG, name
+    assert call(dq=FAKE + 8) == B.DSA_ERR_INVALID_ARG  # misaligned
+    assert call(ws=None) == B.DSA_ERR_WORKSPACE
+    # D and lse2 [1, 4, 1024] fp32, then 2 x 16 bitmaps of ceil(2 * 16 / 32) = 1 word
+    need = 256 + 2 * 16384 + 256
+    assert need <= B.dsa_workspace_size(p)
+    assert call(ws_bytes=need - 1) == B.DSA_ERR_WORKSPACE
