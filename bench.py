@@ -461,6 +461,8 @@ def run_decode(args, w):
     from dynamic_block_sparse_02_b200.attention import BlockSparseAttention
 
     rank, world, local = dist_env()
+    if rank != 0:
+        return 0  # a single-GPU measurement: under torchrun rank 0 runs it alone
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     length = w.N
@@ -564,6 +566,8 @@ def run_backward(args, w):
     from dynamic_block_sparse_02_b200.attention import BlockSparseAttention
 
     rank, world, local = dist_env()
+    if rank != 0:
+        return 0  # a single-GPU measurement: under torchrun rank 0 runs it alone
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     x = W.make_inputs(w, seed=rank_seed(rank))
