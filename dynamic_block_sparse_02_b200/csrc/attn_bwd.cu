@@ -159,23 +159,26 @@ __global__ void __launch_bounds__(BwdCfg<BS, D>::kThreads) bwd_dq_kernel(BwdArgs
   const int bh = b * a.Hq + h;
   const size_t row_id = (size_t)bh * a.nb + i;
 
-  if (tid == 0) {
+  // kept list -> shared memory, 32 entries per step by warp 0, dropping
+  // out-of-range entries (flagged)
+  if (warp == 0) {
     int n = a.cnt[row_id];
     if (n < 0 || n > a.W) {
-      raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnBwd, (int)row_id, n);
+      if (lane == 0) raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnBwd, (int)row_id, n);
       n = n < 0 ? 0 : a.W;
     }
     const int32_t* lst = a.idx + row_id * a.W;
     int m = 0;
-    for (int t = 0; t < n; ++t) {
-      const int j = lst[t];
-      if (j < 0 || j > i) {
-        raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnBwd, (int)row_id, j);
-        continue;
-      }
-      sList[m++] = j;
+    for (int t0 = 0; t0 < n; t0 += 32) {
+      const int t = t0 + lane;
+      const int j = t < n ? lst[t] : 0;
+      const bool bad = t < n && (j < 0 || j > i);
+      if (bad) raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnBwd, (int)row_id, j);
+      const uint32_t keep = __ballot_sync(0xffffffffu, t < n && !bad);
+      if ((keep >> lane) & 1u) sList[m + __popc(keep & ((1u << lane) - 1u))] = j;
+      m += __popc(keep);
     }
-    sCount = m;
+    if (lane == 0) sCount = m;
   }
   __syncthreads();
   const int n_kept = sCount;
