@@ -38,7 +38,7 @@ from dynamic_block_sparse_02_b200 import workloads as W  # noqa: E402
 METRIC = "sparse-attn prefill tokens/s at 32K; effective TFLOP/s vs bf16 tensor peak"
 DEFAULT_WORKLOAD = "32k-gqa"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-ATTN_SOURCES = ("attn_tc.cu", "attn_mma.cu")
+ATTN_SOURCES = ("attn_tc.cu",)  # the kernel whose DRAM traffic profiles/attn_traffic.json records
 SELECT_MODES = {"topk": 0, "group": 1, "threshold": 2}
 
 
@@ -435,7 +435,8 @@ def run_ours(args, w):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config_dict(w),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": recorded_traffic(w.name),
+                     "frac": achieved / peak,
+                     "traffic": recorded_traffic(w.name) if args.attn_kernel in (0, 1) else None,
                      "kernel": "sparse attention (dsa_sparse_attn_fwd)",
                      "peak_kind": f"{peak_kind} bf16 dense, sustained",
                      "frac_of_burst": achieved / float(peaks["bf16_tflops"])},
