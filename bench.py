@@ -73,6 +73,10 @@ def whole_job_tokens_per_s(tokens_per_rank_step: int, world: int, steps: int, ma
     return tokens_per_rank_step * world * steps / (max_ms / 1e3)
 
 
+# 148 SMs x 128 fp32 lanes x 2 FLOP per FMA x 1965 MHz (the part's maximum SM clock)
+FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def kept_flops(cnt_sum: int, block: int, d: int) -> float:
     """Algorithmic FLOPs of the attention step: 4 * bs^2 * d per kept block
     (Q K^T and P V, full tiles, diagonal tile counted in full)."""
@@ -322,6 +326,8 @@ def run_ours(args, w):
     if status != B.DSA_OK:
         raise RuntimeError("device error during warm-up: " + B.status_string(status))
     kept = int(cnt.sum().item())
+    # rows whose kept list holds their own (diagonal) block
+    diag = int((idx == torch.arange(w.nb, device=dev, dtype=idx.dtype).view(1, 1, -1, 1)).any(-1).sum().item())
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
@@ -424,6 +430,7 @@ def run_ours(args, w):
     achieved = flops / (att_avg / 1e3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
     sel_gbs = select_bytes(w) / (sel_avg / 1e3) / 1e9
+    score_flop = 2.0 * w.d * w.B * w.Hq * w.nb * (w.nb + 1) / 2
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         est, desc, spent = oracle_sample(w, x, kph, budget_s=args.cpu_budget)
@@ -441,8 +448,15 @@ def run_ours(args, w):
                      "peak_kind": f"{peak_kind} bf16 dense, sustained",
                      "frac_of_burst": achieved / float(peaks["bf16_tflops"])},
         "select": {"ms": sel_avg, "algorithmic_bytes": select_bytes(w), "GBps": sel_gbs,
-                   "frac_hbm": sel_gbs / float(peaks["hbm_gbs"]), "bound": "hbm"},
+                   "frac_hbm": sel_gbs / float(peaks["hbm_gbs"]), "bound": "hbm",
+                   "frac_spec_8tbs": sel_gbs / 8000.0,
+                   # the fp32 block-score products (j <= i) against the nominal fp32 FMA rate
+                   "score_gflop": score_flop / 1e9,
+                   "score_tflops_at_select_time": score_flop / (sel_avg / 1e3) / 1e12,
+                   "fp32_fma_peak_tflops_nominal": FP32_FMA_PEAK_TFLOPS},
         "attention_ms": att_avg,
+        "attention_tokens_per_s": tokens * world / (att_avg / 1e3),
+        "effective_tflops_diag_half": kept_flops(1, w.block, w.d) * (kept - 0.5 * diag) / (att_avg / 1e3) / 1e12,
         "kept_blocks_per_step": kept,
         "effective_tflops": achieved,
         "cpu_baseline": cpu,
