@@ -33,6 +33,14 @@ What is computed, and where the pages say so:
   1/sqrt(d_k), then the product with V). Query head h reads KV head
   h // (Hq/Hkv) (GQA sharing; zblog post, section on speculative decoding,
   GQA/MQA remark).
+* Decode (see decode): one query token against a KV cache, its own block
+  scored by the mean of its present keys, the prefill rules on that row.
+* Backward (see sparse_attention_backward): the exact gradients of the
+  attention over the kept blocks with the lists held fixed.
+
+Every function here is pinned by tests/test_oracle_pins.py against facts
+independent of it (hand-built closed forms, brute force, PyTorch's textbook
+attention and its autograd, central differences, invariants).
 
 Everything is fp64 except the single fp32 rounding of the scores used for
 ranking. The softmax is the exact two-pass form (row max, then the sum of
