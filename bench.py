@@ -112,6 +112,21 @@ def attn_source_sha() -> str:
     return h.hexdigest()[:16]
 
 
+def recorded_decode_traffic(workload: str, select_mode: str):
+    """DRAM bytes of one decode step (both kernels) from the committed ncu
+    summary, or None when csrc/decode.cu has changed since it was captured."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "decode_traffic.json")) as f:
+            rec = json.load(f)
+        src = os.path.join(ROOT, "dynamic_block_sparse_02_b200", "csrc", "decode.cu")
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except Exception:
+        return None
+    if rec.get("source_sha") != sha or rec.get("workload") != workload or rec.get("select_mode") != select_mode:
+        return None
+    return rec.get("dram_bytes_per_step")
+
+
 def recorded_traffic(workload: str):
     """DRAM bytes per attention launch from the committed ncu summary, or None
     when the attention kernel's source has changed since it was captured."""
@@ -586,7 +601,8 @@ def run_decode(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
-                     "frac": gbs / float(peaks["hbm_gbs"]), "traffic": None,
+                     "frac": gbs / float(peaks["hbm_gbs"]),
+                     "traffic": recorded_decode_traffic(w.name, args.select_mode),
                      "kernel": "decode (dsa_decode_fwd)", "peak_kind": f"{peak_kind} copy bandwidth",
                      "algorithmic_bytes": nbytes},
         "cpu_baseline": cpu,
