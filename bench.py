@@ -205,59 +205,52 @@ class ClockSampler:
 # CPU baseline: the oracle on a bounded sample of the workload
 # ---------------------------------------------------------------------------
 
-def blas_threads() -> int:
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:
-        return 1
+def oracle_sample(w, x, kph, budget_s: float, seed: int = 0, workers=None):
+    """Time the oracle on a bounded sample on the host cores.
 
-
-def oracle_sample(w, x, kph, budget_s: float, seed: int = 0):
-    """Time the oracle on a bounded sample; return (estimated s per full step, description).
-
-    Sample: pooling of all of K plus the pooled Q, scores and selection of the
-    query heads of one KV group; then attention over query blocks of those
-    heads in a seeded random order until ``budget_s`` seconds have passed.
-    The full-step estimate scales selection by Hq / group and attention by
-    (kept blocks of the workload) / (kept blocks processed).
+    Returns (estimated seconds per full step, description, wall seconds spent,
+    cores used). All host cores run oracle workers (one BLAS thread each):
+    pooling, scores and selection of every (batch, KV head) group are timed in
+    full, one group per task; then attention runs over rounds of seeded random
+    query blocks until ``budget_s`` seconds have passed, and its time is
+    scaled by (kept blocks of the workload) / (kept blocks processed).
     """
-    import oracle
-    g = w.group
-    t0 = time.perf_counter()
-    kp = oracle.pool_blocks(x["k"][:, :1], w.block)
-    qp = oracle.pool_blocks(x["q"][:, :g], w.block)
-    s = oracle.block_scores(qp, kp)
-    k = kph[:g] if kph is not None else w.k_free
-    idx, cnt = oracle.select_blocks(s, k, w.local_window, w.n_sink,
-                                    width=min(w.nb, (max(kph) if kph is not None else w.k_free)
-                                              + w.local_window + w.n_sink))
-    t_sel = time.perf_counter() - t0
-    # pooling of Q and K for the remaining heads is part of the full step too
-    t_sel_full = t_sel * (w.Hq / g)
-    rng = np.random.default_rng(seed)
-    order = [(0, h, i) for h in range(g) for i in range(w.nb)]
-    rng.shuffle(order)
-    done, blocks = 0, 0
-    t1 = time.perf_counter()
-    while done < len(order) and time.perf_counter() - t1 < budget_s:
-        chunk = order[done:done + 8]
-        oracle.sparse_attention(x["q"][:, :g], x["k"][:, :1], x["v"][:, :1], idx, cnt, w.block,
-                                items=chunk)
-        blocks += int(sum(cnt[b, h, i] for (b, h, i) in chunk))
-        done += len(chunk)
-    t_att = time.perf_counter() - t1
-    total_blocks = float(cnt.sum()) * (w.B * w.Hq / g)
-    est = t_sel_full + t_att * total_blocks / max(blocks, 1)
-    desc = (f"{w.name}: pooling/scores/selection of {g} query heads (one KV group) timed in full "
-            f"and scaled x{w.Hq // g}; attention on {done} seeded random query blocks "
-            f"({blocks} kept key blocks) timed and scaled to all {int(total_blocks)} kept blocks")
-    return est, desc, t_sel + t_att
+    from oracle.parallel import OraclePool
+    width = min(w.nb, (max(kph) if kph is not None else w.k_free) + w.local_window + w.n_sink)
+    k = kph if kph is not None else w.k_free
+    with OraclePool(dict(q=x["q"], k=x["k"], v=x["v"]), workers=workers) as pool:
+        t0 = time.perf_counter()
+        idx, cnt = pool.select(w.B, w.Hkv, w.group, w.block, k, w.local_window, w.n_sink, width)
+        t_sel = time.perf_counter() - t0
+        pool.put("idx", idx)
+        pool.put("cnt", cnt)
+        rng = np.random.default_rng(seed)
+        order = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.nb)]
+        rng.shuffle(order)
+        per_round = 2 * pool.workers
+        done, blocks, t_att = 0, 0, 0.0
+        while done < len(order) and t_att < budget_s:
+            chunk = order[done:done + per_round]
+            t_att += pool.timed_attention(chunk, w.block)
+            blocks += int(sum(cnt[it] for it in chunk))
+            done += len(chunk)
+        cores = pool.workers
+    total_blocks = float(cnt.sum())
+    est = t_sel + t_att * total_blocks / max(blocks, 1)
+    desc = (f"{w.name}: pooling/scores/selection of all {w.B * w.Hkv} (batch, KV head) groups timed "
+            f"in full ({t_sel:.1f} s); attention on {done} seeded random query blocks ({blocks} kept "
+            f"key blocks, {t_att:.1f} s) scaled to all {int(total_blocks)} kept blocks; "
+            f"{cores} worker processes, one BLAS thread each")
+    return est, desc, t_sel + t_att, cores
 
 
 def run_reference(args, w):
-    """The --impl reference arm: the oracle as it stands, on host cores."""
+    """The --impl reference arm: the oracle as it stands, on host cores.
+
+    Each step is a bounded sample of the workload (see oracle_sample);
+    ms_per_step is that sample's measured wall time, and value is the
+    workload's tokens divided by the full step time extrapolated from it.
+    """
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
@@ -265,20 +258,22 @@ def run_reference(args, w):
     kph = None if kph is None else [int(t) for t in kph]
     x = W.make_inputs(w, seed=rank_seed(0))
     for _ in range(args.warmup):
-        oracle_sample(w, x, kph, budget_s=1.0)
-    ests, desc = [], ""
+        oracle_sample(w, x, kph, budget_s=min(1.0, args.ref_budget))
+    ests, walls, desc, cores = [], [], "", 1
     for s in range(args.steps):
-        est, desc, _ = oracle_sample(w, x, kph, budget_s=args.ref_budget, seed=s)
+        est, desc, wall, cores = oracle_sample(w, x, kph, budget_s=args.ref_budget, seed=s)
         ests.append(est)
+        walls.append(wall)
     est = statistics.median(ests)
     tokens = w.B * w.N
     value = tokens / est
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(walls) * 1e3,
+        "ms_per_full_step_extrapolated": est * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_dict(w),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -286,12 +281,27 @@ def run_reference(args, w):
     return 0
 
 
+L2_BYTES = 126 << 20          # B200 L2
+FLUSH_BYTES = 256 << 20       # written between timed steps when the inputs fit in L2
+
+
+def input_bytes(w) -> int:
+    return w.B * (w.Hq + 2 * w.Hkv) * w.N * w.d * 2
+
+
+def needs_flush(w) -> bool:
+    """Inputs below twice the L2 size would partly stay in L2 from one step to the next."""
+    return input_bytes(w) < 2 * L2_BYTES
+
+
 def config_dict(w):
+    mb = input_bytes(w) / 1e6
+    l2 = ("L2 flushed before every timed step (%d MB written; Q+K+V = %.1f MB); "
+          "ms_per_step sums the steps' own event times" % (FLUSH_BYTES >> 20, mb)
+          if needs_flush(w) else "inputs larger than L2: Q+K+V = %.0f MB per step > 126 MB" % mb)
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
             "block": w.block, "k_free": w.k_free, "local_window": w.local_window,
-            "n_sink": w.n_sink,
-            "l2": "inputs larger than L2: Q+K+V = %.0f MB per step > 126 MB"
-                  % ((w.B * (w.Hq + 2 * w.Hkv) * w.N * w.d * 2) / 1e6)}
+            "n_sink": w.n_sink, "l2": l2}
 
 
 # ---------------------------------------------------------------------------
@@ -351,9 +361,12 @@ def run_ours(args, w):
         sampler.start()
     if world > 1:
         dist.barrier()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if needs_flush(w) else None
     torch.cuda.synchronize(dev)
     with torch.cuda.stream(stream):
         for s in range(K):
+            if flush is not None:
+                flush.fill_(s & 0xff)
             ev[s][0].record(stream)
             select()
             ev[s][1].record(stream)
@@ -367,7 +380,10 @@ def run_ours(args, w):
     if status != B.DSA_OK:
         raise RuntimeError("device error during timing: " + B.status_string(status))
 
-    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    if flush is None:
+        total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    else:  # the flushes between steps are not part of the steps
+        total_ms = sum(e[0].elapsed_time(e[2]) for e in ev)
     sel_ms = [e[0].elapsed_time(e[1]) for e in ev]
     att_ms = [e[1].elapsed_time(e[2]) for e in ev]
     max_total = reduce_max(total_ms, dev)
@@ -443,14 +459,15 @@ def run_ours(args, w):
     sel_avg = statistics.mean(sel_ms)
     flops = kept_flops(kept, w.block, w.d)
     achieved = flops / (att_avg / 1e3) / 1e12
-    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    # the attention kernel runs as millisecond launches: the burst peak applies
+    peak = float(peaks["bf16_tflops"])
     sel_gbs = select_bytes(w) / (sel_avg / 1e3) / 1e9
     score_flop = 2.0 * w.d * w.B * w.Hq * w.nb * (w.nb + 1) / 2
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        est, desc, spent = oracle_sample(w, x, kph, budget_s=args.cpu_budget)
-        cpu = {"value": tokens / est, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": desc + f" ({spent:.1f} s of CPU work)"}
+        est, desc, spent, cores = oracle_sample(w, x, kph, budget_s=args.cpu_budget)
+        cpu = {"value": tokens / est, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": desc + f" ({spent:.1f} s wall)"}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": max_total / K, "higher_is_better": True,
@@ -460,8 +477,9 @@ def run_ours(args, w):
                      "frac": achieved / peak,
                      "traffic": recorded_traffic(w.name) if args.attn_kernel in (0, 1) else None,
                      "kernel": "sparse attention (dsa_sparse_attn_fwd)",
-                     "peak_kind": f"{peak_kind} bf16 dense, sustained",
-                     "frac_of_burst": achieved / float(peaks["bf16_tflops"])},
+                     "peak_kind": f"{peak_kind} bf16 dense, burst",
+                     "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained",
+                                                                     peaks["bf16_tflops"]))},
         "select": {"ms": sel_avg, "algorithmic_bytes": select_bytes(w), "GBps": sel_gbs,
                    "frac_hbm": sel_gbs / float(peaks["hbm_gbs"]), "bound": "hbm",
                    "frac_spec_8tbs": sel_gbs / 8000.0,
@@ -581,17 +599,19 @@ def run_decode(args, w):
     cpu = None
     if not args.no_cpu_baseline:
         import oracle
-        t0 = time.perf_counter()
-        steps = 0
-        while True:  # whole decode steps until about cpu_budget seconds of CPU work
-            oracle.decode(qtok_h, x["k"], x["v"], length, w.block, w.k_free, w.local_window, w.n_sink,
-                          mode=args.select_mode, tau=args.tau if args.select_mode == "threshold" else 0.0)
-            steps += 1
-            if time.perf_counter() - t0 >= args.cpu_budget or steps >= 200:
-                break
-        spent = time.perf_counter() - t0
-        cpu = {"value": steps * w.B / spent, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{steps} full decode steps ({spent:.1f} s of CPU work)"}
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(1):  # one core: the step is one row per head
+            t0 = time.perf_counter()
+            steps = 0
+            while True:  # whole decode steps until about cpu_budget seconds of CPU work
+                oracle.decode(qtok_h, x["k"], x["v"], length, w.block, w.k_free, w.local_window, w.n_sink,
+                              mode=args.select_mode, tau=args.tau if args.select_mode == "threshold" else 0.0)
+                steps += 1
+                if time.perf_counter() - t0 >= args.cpu_budget or steps >= 200:
+                    break
+            spent = time.perf_counter() - t0
+        cpu = {"value": steps * w.B / spent, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"{steps} full decode steps on one core, BLAS on one thread ({spent:.1f} s)"}
     cfg = config_dict(w)
     cfg["l2"] = ("L2 flushed before every timed step: 256 MB write, then 256 MB read "
                  "(clean cold L2); ms_per_step_dirty_l2 = the same after the write alone")
@@ -672,17 +692,22 @@ def run_backward(args, w):
     peaks, peak_kind = load_peaks()
     flops = backward_flops(kept, w.block, w.d)
     tfs = flops / (step_ms / 1e3) / 1e12
-    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    peak = float(peaks["bf16_tflops"])  # millisecond launches: the burst peak applies
     cpu = None
     if not args.no_cpu_baseline:
-        import oracle
+        from oracle.parallel import OraclePool
         idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
         items = [(0, h, i) for h in range(w.Hq) for i in range(w.nb - 1, -1, -97)][:args.bwd_sample]
-        t0 = time.perf_counter()
-        oracle.sparse_attention_backward(x["q"], x["k"], x["v"], do_h, idx_h, cnt_h, w.block, items=items)
-        spent = time.perf_counter() - t0
-        cpu = {"value": len(items) * w.block / spent, "unit": "tokens/s", "cores": blas_threads(),
-               "kind": "oracle", "sample": f"{len(items)} query blocks of the workload ({spent:.1f} s)"}
+        with OraclePool(dict(q=x["q"], k=x["k"], v=x["v"], dout=do_h, idx=idx_h, cnt=cnt_h)) as pool:
+            t0 = time.perf_counter()
+            pool.backward(items, w.block)
+            spent = time.perf_counter() - t0
+            cores = pool.workers
+        share = float(sum(cnt_h[it] for it in items)) / float(cnt_h.sum())
+        cpu = {"value": w.B * w.N * share / spent, "unit": "tokens/s", "cores": cores,
+               "kind": "oracle",
+               "sample": f"{len(items)} query blocks of the workload ({share:.3%} of its kept blocks, "
+                         f"{spent:.1f} s wall on {cores} worker processes), scaled by kept blocks"}
     cfg = config_dict(w)
     cfg["l2"] = "inputs larger than L2 (q, dout, out 268 MB each), no flush"
     cfg["selection"] = "the forward's own top-k lists"
@@ -692,7 +717,8 @@ def run_backward(args, w):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
         "roofline": {"bound": "tensor", "achieved": tfs, "peak": peak, "unit": "TFLOP/s", "frac": tfs / peak,
                      "traffic": None, "kernel": "backward step (prep, colbits, dq, dkv)",
-                     "peak_kind": f"{peak_kind} sustained bf16", "algorithmic_flops": flops},
+                     "peak_kind": f"{peak_kind} bf16 dense, burst", "algorithmic_flops": flops,
+                     "frac_of_sustained": tfs / float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))},
         "kept_blocks": kept,
         "cpu_baseline": cpu,
         "gpu_launches": 4 * args.steps,

@@ -3,6 +3,7 @@
 // synchronises the host, except dsa_check_status, which synchronises on
 // purpose to read the device error flag.
 #include <cmath>
+#include <cuda.h>
 #include <cstring>
 #include <mutex>
 
@@ -192,23 +193,64 @@ static __device__ __align__(256) unsigned char g_select_scratch[kStaticScratchBy
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {nullptr};
+struct ScratchAddr {
+  unsigned long long ctx_id;  // unique id of the CUDA context the address belongs to
+  void* addr;
+};
+ScratchAddr g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_select_scratch on the current device. The first call on
-// a device looks it up with cudaGetSymbolAddress (which may load the module on
-// that device); later calls return the cached address.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current CUDA context (driver entry points
+// through the runtime, so the library needs no link against libcuda).
+// Returns false when there is no current context yet.
+bool current_ctx_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (get_current == nullptr || get_id == nullptr) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess)
+      return false;
+    get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+    get_id = reinterpret_cast<CtxGetIdFn>(f2);
+  }
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_select_scratch in the current device's context. The
+// first call in a context looks it up with cudaGetSymbolAddress (which may
+// load the module into that context); later calls in the same context return
+// the cached address. The cache is keyed on the context's unique id, so a
+// context that was destroyed and re-created (cudaDeviceReset, a primary
+// context released and retained again) gets a fresh lookup, never the old
+// context's address.
 dsa_status select_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return DSA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* addr = nullptr;
-    if (cudaGetSymbolAddress(&addr, g_select_scratch) != cudaSuccess || addr == nullptr)
-      return DSA_ERR_CUDA;
-    g_scratch_addr[dev] = addr;
+  unsigned long long id = 0;
+  const bool have_id = current_ctx_id(&id);
+  if (have_id && g_scratch_addr[dev].addr != nullptr && g_scratch_addr[dev].ctx_id == id) {
+    *out = g_scratch_addr[dev].addr;
+    return DSA_OK;
   }
-  *out = g_scratch_addr[dev];
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_select_scratch) != cudaSuccess || addr == nullptr)
+    return DSA_ERR_CUDA;
+  // the lookup has made a context current if none was
+  if (!current_ctx_id(&id)) return DSA_ERR_CUDA;
+  g_scratch_addr[dev].ctx_id = id;
+  g_scratch_addr[dev].addr = addr;
+  *out = addr;
   return DSA_OK;
 }
 

@@ -111,9 +111,15 @@ typedef enum dsa_attn_kernel {
  *                      k_per_head == NULL and Hq/Hkv <= 32.
  *   select_tau       : DSA_SELECT_THRESHOLD: the threshold tau, 0 < tau <= 1;
  *                      other modes: must be 0. The block probabilities are
- *                      computed in fp32 (exp2 of scale * log2(e) * (s - max)),
- *                      so a block within ~1e-6 relative of the threshold may
- *                      fall on either side of it.
+ *                      computed in fp32 (exp2 of c2 * (s - max) over their
+ *                      fp32 sum, c2 = scale * log2(e)), so a block j of query
+ *                      block i whose exact probability p_j is within
+ *                      delta_j * tau of tau may fall on either side, with
+ *                        eps_j   = (block + d) 2^-24 sum_d mean|q_d| mean|k_jd|
+ *                                  (fp32 error bound of the score s(i, j);
+ *                                  mean|.| over the block's rows),
+ *                        eta_j   = c2 (eps_j + max eps) + 2^-23 c2 |s_j - max s|,
+ *                        delta_j = ln2 (eta_j + max eta) + (i + 5) 2^-24 + 2^-21.
  */
 typedef struct dsa_params {
   int B, Hq, Hkv, N, d;
@@ -179,9 +185,12 @@ dsa_status dsa_select_blocks(const dsa_params *p, const dsa_bf16 *q, const dsa_b
  *     needs to start at zero. A problem whose pooled Qp and Kp (fp32,
  *     B*(Hq+Hkv)*nb*d*4 bytes, each part rounded up to 256) exceed 16 MiB gets
  *     DSA_ERR_WORKSPACE and launches nothing.
- *   - Set-up: the first call on a device looks the array's address up
- *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture on the device.
+ *   - Set-up: the first call in a device's CUDA context looks the array's
+ *     address up (cudaGetSymbolAddress, with that device current) and caches
+ *     it per context; make that first call before any stream capture on the
+ *     device. A context that is destroyed and created again (e.g. after
+ *     cudaDeviceReset) gets a new lookup on its first call; the array's
+ *     contents do not survive the reset.
  *   - Overlapping calls on one device (two streams, two host threads) share
  *     the array and race: order them (one stream, or events).
  *   - Arguments, outputs and argument errors as dsa_select_blocks; the result

@@ -1,8 +1,20 @@
 """GPU parity of the threshold selection rule (forced blocks plus the blocks
 whose share of the softmax over the row's block logits is >= tau, at most k)
-against the fp64 oracle, through the C ABI. A block whose oracle probability
-lies within 1e-4 (relative) of tau may fall on either side on the GPU (fp32
-probabilities), and the usual near-tie rule applies at the k-th score.
+against the fp64 oracle, through the C ABI.
+
+A block may fall on the other side of tau on the GPU only when its oracle
+probability p_j is within delta_j * tau of tau, delta_j being the bound on the
+relative error of the GPU's fp32 probability (the same bound include/dsa.h
+states for DSA_SELECT_THRESHOLD):
+  eps_j   = (bs + d) * 2^-24 * sum_d mean|q_d| * mean|k_jd|   fp32 error of s(i, j)
+            (block means of bs terms, then a d-term dot product; mean|.| over
+            the block's rows)
+  eta_j   = c2 * (eps_j + max eps) + 2^-23 * c2 * |s_j - max s|   exponent error
+  delta_j = ln2 * (eta_j + max eta) + (i + 5) * 2^-24 + 2^-21
+with c2 = scale * log2(e); the ln2 terms are the errors of 2^x from errors in x
+(for the block and for the normaliser's largest term), (i + 5) 2^-24 the fp32
+sum of i + 1 terms and the products, 2^-21 the exp2 approximation. The usual
+near-tie rule applies at the k-th score.
 """
 import numpy as np
 import pytest
@@ -18,7 +30,22 @@ from parity import TIE_REL, assert_attention_close, dev_bf16, dev_i32
 pytestmark = pytest.mark.gpu
 
 THR = B.DSA_SELECT_THRESHOLD
-BOUNDARY_REL = 1e-4
+U32 = 2.0 ** -24
+
+
+def block_abs_means(bits, block):
+    """mean over each block's rows of |x| (fp64) [B, H, nb, d]."""
+    x = np.abs(W.bf16_bits_to_f32(bits).astype(np.float64))
+    Bn, H, N, d = x.shape
+    return x.reshape(Bn, H, N // block, block, d).mean(axis=3)
+
+
+def prob_error_bound(aq, ak, s_row, i, block, d, c2):
+    """delta_j of the module docstring for every causal block j of one row."""
+    eps = (block + d) * U32 * (ak[:i + 1] @ aq)
+    m = np.max(s_row[:i + 1])
+    eta = c2 * (eps + eps.max()) + 2 * U32 * c2 * np.abs(s_row[:i + 1] - m)
+    return np.log(2.0) * (eta + eta.max()) + (i + 5) * U32 + 2.0 ** -21
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -28,11 +55,13 @@ def need_cuda():
     torch.cuda.set_device(0)
 
 
-def compare_threshold(idx_g, cnt_g, idx_r, cnt_r, s64, tau, k, w, ns, scale):
+def compare_threshold(idx_g, cnt_g, idx_r, cnt_r, s64, tau, k, w, ns, scale, aq, ak, block, d):
     """Unexcused row mismatches: every block in the symmetric difference must
-    sit at the threshold (probability within BOUNDARY_REL of tau) or tie with
-    the k-th candidate's score (TIE_REL)."""
+    sit at the threshold (|p_j - tau| <= delta_j * tau) or tie with the k-th
+    candidate's score (TIE_REL)."""
     B_, Hq, nb, _ = idx_r.shape
+    g = Hq // ak.shape[1]
+    c2 = scale * np.log2(np.e)
     bad = []
     for b in range(B_):
         for h in range(Hq):
@@ -49,8 +78,9 @@ def compare_threshold(idx_g, cnt_g, idx_r, cnt_r, s64, tau, k, w, ns, scale):
                 cand = [j for j in range(i + 1) if j not in forced]
                 srt = sorted(cand, key=lambda j: (-float(np.float32(s64[b, h, i, j])), j))
                 kth = s64[b, h, i, srt[min(k, len(srt)) - 1]] if srt and k > 0 else None
+                delta = prob_error_bound(aq[b, h, i], ak[b, h // g], s64[b, h, i], i, block, d, c2)
                 for j in set(g) ^ set(r):
-                    at_bar = abs(p[j] - tau) <= BOUNDARY_REL * tau
+                    at_bar = abs(p[j] - tau) <= delta[j] * tau
                     at_cut = kth is not None and abs(s64[b, h, i, j] - kth) <= TIE_REL * max(
                         abs(s64[b, h, i, j]), abs(kth))
                     if j in forced or not (at_bar or at_cut):
@@ -81,7 +111,8 @@ def test_threshold_selection_parity(name):
     q, kk, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
     idx, cnt = att.select_blocks(q, kk)
     idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
-    bad = compare_threshold(idx_h, cnt_h, idx_r, cnt_r, s64, tau, k, lw, ns, scale)
+    aq, ak = block_abs_means(x["q"], bs), block_abs_means(x["k"], bs)
+    bad = compare_threshold(idx_h, cnt_h, idx_r, cnt_r, s64, tau, k, lw, ns, scale, aq, ak, bs, d)
     assert not bad, bad[:5]
     # the rule is doing something: some rows keep fewer than k free blocks
     full = np.array([min(i + 1, k + len(oracle.forced_set(i, lw, ns))) for i in range(w.nb)])
