@@ -15,6 +15,7 @@ struct WsHeader {
   int status;           // first device-side error (dsa_status value), 0 = none
   int detail[3];        // kernel id and a coordinate of the first error
   unsigned int work[8]; // work counters of persistent kernels (reset per call)
+  unsigned long long wait_limit_ns;  // limit of the kernels' bounded waits; 0 = default (2 s)
 };
 constexpr size_t kHeaderBytes = 256;
 static_assert(sizeof(WsHeader) <= kHeaderBytes, "header too large");
