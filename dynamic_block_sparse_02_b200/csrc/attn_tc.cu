@@ -1,6 +1,6 @@
 // Block-sparse causal attention forward (step 4) on the 5th-generation tensor
 // cores (tcgen05 + TMEM + TMA), for 32x32 and 64x64 blocks and head dim 64
-// or 128 (one kernel template; 128x128 blocks run in attn_tc_rows.cu).
+// or 128 (one kernel template; 128x128 blocks run in attn_tc128.cu).
 //
 // What it computes is the same as the warp-MMA kernel: for every query block
 // i of (b, query head h), softmax(Q K^T * scale) V over the kept key blocks
@@ -786,13 +786,14 @@ bool attn_tc_supported(const Shape& s) {
   // TMA row coordinates are 32-bit
   const unsigned long long rows = (unsigned long long)s.B * s.Hq * s.N;
   if (rows >= (1ull << 31) || encode_fn() == nullptr) return false;
-  return (s.bs == 32 || s.bs == 64) && (s.d == 64 || s.d == 128);
+  return (s.bs == 32 || s.bs == 64 || s.bs == 128) && (s.d == 64 || s.d == 128);
 }
 
 cudaError_t launch_attn_tc(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const __nv_bfloat16* v, const int32_t* idx, const int32_t* cnt,
                            __nv_bfloat16* out, float* lse, WsHeader* hdr, cudaStream_t st) {
   if (!attn_tc_supported(s)) return cudaErrorNotSupported;
+  if (s.bs == 128) return launch_attn_tc128(s, q, k, v, idx, cnt, out, lse, hdr, st);
   if (s.bs == 64 && s.d == 128) return launch_shape<64, 128>(s, q, k, v, idx, cnt, out, lse, hdr, st);
   if (s.bs == 64 && s.d == 64) return launch_shape<64, 64>(s, q, k, v, idx, cnt, out, lse, hdr, st);
   if (s.bs == 32 && s.d == 128) return launch_shape<32, 128>(s, q, k, v, idx, cnt, out, lse, hdr, st);

@@ -130,6 +130,10 @@ cudaError_t launch_attn_mma(const Shape& s, const __nv_bfloat16* q, const __nv_b
                             const __nv_bfloat16* v, const int32_t* idx, const int32_t* cnt,
                             __nv_bfloat16* out, float* lse, WsHeader* hdr, cudaStream_t st);
 bool attn_tc_supported(const Shape& s);
+// 128x128 blocks (attn_tc128.cu); called by launch_attn_tc.
+cudaError_t launch_attn_tc128(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                              const __nv_bfloat16* v, const int32_t* idx, const int32_t* cnt,
+                              __nv_bfloat16* out, float* lse, WsHeader* hdr, cudaStream_t st);
 cudaError_t launch_attn_tc(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const __nv_bfloat16* v, const int32_t* idx, const int32_t* cnt,
                            __nv_bfloat16* out, float* lse, WsHeader* hdr, cudaStream_t st);

@@ -88,7 +88,7 @@ __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, vo
   }
 }
 
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile CtaFlags* f,
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile CtaFlags* f,
                                             WsHeader* hdr, int kernel, int where) {
   return mbar_wait_spin<false>(bar, parity, f, hdr, kernel, where);
 }
@@ -122,7 +122,7 @@ __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, WsHead
 // Waits for a barrier phase that belongs to walk step n. Returns 1 when the
 // phase completed, 0 when the walk has fewer than n + 1 steps (the step and
 // its phase never come), -1 when the kernel is aborting or the wait timed out.
-__device__ __noinline__ int step_wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* total,
+static __device__ __noinline__ int step_wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* total,
                                            uint32_t n, volatile CtaFlags* f, WsHeader* hdr,
                                            int kernel, int where) {
   const unsigned long long t0 = now_ns();

@@ -108,7 +108,7 @@ def test_small_case_all_steps(name):
 
 
 def tc_supported(w):
-    return w.block in (32, 64) and w.d in (64, 128)
+    return w.block in (32, 64, 128) and w.d in (64, 128)
 
 
 def test_explicit_tcgen05_kernel_or_unsupported():
