@@ -59,11 +59,11 @@ using namespace tc;
 constexpr int kChunk = 128;    // keys per S^T tile
 constexpr int kThreads = 384;
 constexpr int kStreams = 2;
-constexpr int kPTiles = 3;     // P tiles shared by the streams
 constexpr float kTau = 8.0f;   // rescale threshold (log2 units)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr int kNumBars = 36;
+constexpr int kMaxPT = 6;      // most P tiles of any shape
+constexpr int kNumBars = 50;
 
 // Sizes and shared-memory map for bs x bs blocks and head dim d. Every tile is
 // a stack of 128-byte swizzle atoms [d / 64][rows][128 B] (K-major rows of
@@ -83,18 +83,24 @@ struct Cfg {
   static constexpr int PRow = BS * 2;                // bytes per key row of P^T
   static constexpr int PBytes = kChunk * PRow;
   static constexpr uint32_t PLayout = BS == 64 ? 2u : 4u;  // 128- / 64-byte swizzle
+  // K and V ring stages: 16 KB stages (d = 64) need a deeper ring to hide the
+  // copy latency behind the short steps; 32 KB stages fill shared memory at 2.
+  static constexpr int NSTG = D == 64 ? 4 : 2;
   static constexpr int OffQ = 0;                           // one per stream
-  static constexpr int OffK = OffQ + kStreams * QBytes;    // 2 ring stages
-  static constexpr int OffV = OffK + 2 * KVBytes;          // 2 ring stages
-  static constexpr int OffP = OffV + 2 * KVBytes;          // [kPTiles]
-  static constexpr int OffList = OffP + kPTiles * PBytes;  // [stream][slot][kMaxBlocks] int16
+  static constexpr int OffK = OffQ + kStreams * QBytes;    // NSTG ring stages
+  static constexpr int OffV = OffK + NSTG * KVBytes;       // NSTG ring stages
+  // P tiles shared by the two streams (as many as shared memory holds, <= kMaxPT)
+  static constexpr int PT = (BS == 64 && D == 128) ? 3 : (BS == 64 ? 4 : 6);
+  static constexpr int OffP = OffV + NSTG * KVBytes;       // [PT]
+  static constexpr int OffList = OffP + PT * PBytes;       // [stream][slot][kMaxBlocks] int16
   static constexpr int OffRed = OffList + kStreams * 2 * kMaxBlocks * 2;  // [stream][4][BS] f32
   static constexpr int OffM = OffRed + kStreams * 4 * BS * 4;  // [stream][BS] -(running max)
   static constexpr int OffL = OffM + kStreams * BS * 4;        // [stream][BS] 1 / row sum
   static constexpr int OffA = OffL + kStreams * BS * 4;        // [stream][BS] max increments
   static constexpr int OffBar = OffA + kStreams * BS * 4;      // mbarriers
   static constexpr int OffMisc = OffBar + kNumBars * 8;        // tmem base, item slots, step ids, wait flags
-  static constexpr int SmemBytes = OffMisc + 176 + 1024;       // + alignment slack
+  static constexpr int SmemBytes = OffMisc + 192 + 1024;       // + alignment slack
+  static_assert(PT <= kMaxPT, "P tiles");
   static_assert(QBytes % 1024 == 0 && KVBytes % 1024 == 0 && PBytes % 1024 == 0, "atom alignment");
   static_assert(SmemBytes <= 232448, "shared memory budget");
   // TMEM columns per stream: two S^T buffers and the O^T accumulator.
@@ -113,19 +119,19 @@ enum {
   B_ITEM_EMPTY = 4,   // [2][2]
   B_Q_FULL = 8,       // [2]
   B_Q_EMPTY = 10,     // [2]
-  B_K_FULL = 12,      // [2]
-  B_K_EMPTY = 14,     // [2] spare: a K stage is free once its S^T has completed (S_FULL)
-  B_V_FULL = 16,      // [2]
-  B_V_EMPTY = 18,     // [2] spare: a V stage is free once its PV has completed (P_EMPTY)
-  B_S_FULL = 20,      // [2][2]
-  B_S_FREE = 24,      // [2][2]
-  B_P_FULL = 28,      // [kPTiles]
-  B_P_EMPTY = 31,     // [kPTiles]
-  B_O_DONE = 34       // [2]: the last PV of a stream's item has finished
+  B_S_FULL = 12,      // [2][2]
+  B_S_FREE = 16,      // [2][2]
+  B_P_FULL = 20,      // [PT <= kMaxPT]
+  B_P_EMPTY = 26,     // [PT]
+  B_O_DONE = 32,      // [2]: the last PV of a stream's item has finished
+  B_K_FULL = 34,      // [NSTG <= 4]
+  B_K_EMPTY = 38,     // [NSTG] the S^T that read the stage has completed
+  B_V_FULL = 42,      // [NSTG]
+  B_V_EMPTY = 46      // [NSTG] the PV that read the stage has completed
 };
 
-// P tiles: step n of the (stream, chunk) walk writes tile n % kPTiles, whose
-// previous reader was step n - kPTiles; the S^T issuer publishes each step's
+// P tiles: step n of the (stream, chunk) walk writes tile n % PT, whose
+// previous reader was step n - PT; the S^T issuer publishes each step's
 // index next to its S^T buffer (sStep[stream][buffer]).
 
 struct ItemSlot {
@@ -177,15 +183,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bars = sbase + C::OffBar;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + C::OffMisc);
-  volatile CtaFlags* sFlags = reinterpret_cast<volatile CtaFlags*>(smem + C::OffMisc + 160);
+  volatile CtaFlags* sFlags = reinterpret_cast<volatile CtaFlags*>(smem + C::OffMisc + 176);
   volatile int* sAbort = &sFlags->abort;
   ItemSlot* sItem = reinterpret_cast<ItemSlot*>(smem + C::OffMisc + 16);  // [stream][slot]
   volatile uint32_t* sStep = reinterpret_cast<volatile uint32_t*>(smem + C::OffMisc + 112);  // [stream][S buffer]
   // step count of the whole walk, published by the K producer when it ends
   volatile uint32_t* sTotal = reinterpret_cast<volatile uint32_t*>(smem + C::OffMisc + 8);
   // per K stage and per P tile: stream and position of the step they hold
-  volatile uint32_t* sKMeta = reinterpret_cast<volatile uint32_t*>(smem + C::OffMisc + 128);  // [2]
-  volatile uint32_t* sPMeta = reinterpret_cast<volatile uint32_t*>(smem + C::OffMisc + 136);  // [kPTiles]
+  volatile uint32_t* sKMeta = reinterpret_cast<volatile uint32_t*>(smem + C::OffMisc + 128);  // [NSTG]
+  volatile uint32_t* sPMeta = reinterpret_cast<volatile uint32_t*>(smem + C::OffMisc + 144);  // [PT]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   auto bar = [&](int idx) { return bars + 8u * idx; };
@@ -202,12 +208,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(bar(B_Q_FULL + x), 1);
       mbar_init(bar(B_Q_EMPTY + x), 1);
       mbar_init(bar(B_O_DONE + x), 1);
-      mbar_init(bar(B_K_FULL + x), 1);
-      mbar_init(bar(B_K_EMPTY + x), 1);
-      mbar_init(bar(B_V_FULL + x), 1);
-      mbar_init(bar(B_V_EMPTY + x), 1);
     }
-    for (int t = 0; t < kPTiles; ++t) {
+    for (int u = 0; u < C::NSTG; ++u) {
+      mbar_init(bar(B_K_FULL + u), 1);
+      mbar_init(bar(B_K_EMPTY + u), 1);
+      mbar_init(bar(B_V_FULL + u), 1);
+      mbar_init(bar(B_V_EMPTY + u), 1);
+    }
+    for (int t = 0; t < C::PT; ++t) {
       mbar_init(bar(B_P_FULL + t), 128);
       mbar_init(bar(B_P_EMPTY + t), 1);
     }
@@ -237,11 +245,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       int16_t* const lists = reinterpret_cast<int16_t*>(smem + C::OffList);
       uint32_t gk = 0;
       Pair<uint32_t> gq = {0u, 0u};
-      Pair<uint32_t> gs = {0u, 0u};  // S^T uses per stream, as counted by the S issuer
-      // per K stage u: bit 8u: loaded once; bits 8u+1..: s_full barrier index and
-      // parity of the S^T step that read it (the stage is free once that completes)
-      uint32_t kuse = 0;
-      // bit u set: ring stage u has an issued load; bit 2+u: its phase parity
+      // bit u set: ring stage (or Q buffer) u has an issued load; bit 8+u: its phase parity
       uint32_t lastK = 0, lastQ = 0;
       Pair<int> kvrow = {0, 0};
       Pair<int> nkept = {0, 0};
@@ -308,7 +312,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
                 for (int hh = 0; hh < C::DH; ++hh)
                   tma_load_2d(dq + hh * C::QAtom, &tmQ, 64 * hh, qrow, bar(B_Q_FULL + x));
-                lastQ = (lastQ & ~(5u << x)) | (1u << x) | ((gqx & 1u) << (2 + x));
+                lastQ = (lastQ & ~(0x101u << x)) | (1u << x) | ((gqx & 1u) << (8 + x));
               }
               gq.inc(x);
             }
@@ -325,9 +329,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const int nblk = min(C::NBC, nkept.get(x) - C::NBC * c);
           const int kvr = kvrow.get(x);
           const int16_t* my_list = lists + (2 * x + (wk.t.get(x) & 1)) * kMaxBlocks;
-          const uint32_t ks = gk & 1;
-          const uint32_t prev = (kuse >> (8 * ks)) & 0xffu;
-          if (prev & 1u) ok = ok && mbar_wait(bar(B_S_FULL + (prev >> 2)), (prev >> 1) & 1u, wc, 3);
+          const uint32_t ks = gk % C::NSTG;
+          // the stage's previous tile was read by the S^T of load gk - NSTG
+          if (gk >= (uint32_t)C::NSTG) ok = ok && mbar_wait(bar(B_K_EMPTY + ks), ((gk / C::NSTG) - 1) & 1, wc, 3);
           if (ok) {
             sKMeta[ks] = step_meta(x, c == 0, c == wk.C.get(x) - 1, nblk);
             mbar_expect_tx(bar(B_K_FULL + ks), nblk * BS * D * 2);
@@ -338,14 +342,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               for (int hh = 0; hh < C::DH; ++hh)
                 tma_load_2d(dk + hh * C::KVAtom + bb * BS * 128, &tmK, 64 * hh, row, bar(B_K_FULL + ks));
             }
-            lastK = (lastK & ~(5u << ks)) | (1u << ks) | (((gk >> 1) & 1u) << (2 + ks));
+            lastK = (lastK & ~(0x101u << ks)) | (1u << ks) | (((gk / C::NSTG) & 1u) << (8 + ks));
           }
-          // the S^T step of this K tile writes buffer gs & 1 of stream x
-          const uint32_t gsx = gs.get(x);
-          const uint32_t use = 1u | (((gsx >> 1) & 1u) << 1) | ((uint32_t)(2 * x + (gsx & 1)) << 2);
-          kuse = (kuse & ~(0xffu << (8 * ks))) | (use << (8 * ks));
         }
-        gs.inc(x);
         ++gk;
         ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
         wk.advance(x);
@@ -353,10 +352,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (lane == 0) *sTotal = gk;
       // drain: every issued load has landed before the CTA may exit
       if (lane == 0) {
-        for (int u = 0; u < 2; ++u) {
-          if (lastK & (1u << u)) mbar_drain(bar(B_K_FULL + u), (lastK >> (2 + u)) & 1u, a.hdr, kKernAttnTc, 5);
-          if (lastQ & (1u << u)) mbar_drain(bar(B_Q_FULL + u), (lastQ >> (2 + u)) & 1u, a.hdr, kKernAttnTc, 5);
-        }
+        for (int u = 0; u < C::NSTG; ++u)
+          if (lastK & (1u << u)) mbar_drain(bar(B_K_FULL + u), (lastK >> (8 + u)) & 1u, a.hdr, kKernAttnTc, 5);
+        for (int u = 0; u < kStreams; ++u)
+          if (lastQ & (1u << u)) mbar_drain(bar(B_Q_FULL + u), (lastQ >> (8 + u)) & 1u, a.hdr, kKernAttnTc, 5);
       }
     } else if (warp == 3) {
       // ---------------------------------------------------------------- V producer
@@ -393,10 +392,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const int c = wk.c.get(x);
           const int slot = wk.t.get(x) & 1;
           const int nblk = min(C::NBC, nkept.get(x) - C::NBC * c);
-          const uint32_t vs = gv & 1;
-          // the stage's previous tile belongs to step gv - 2, whose PV also freed its P tile
-          if (gv >= 2)
-            ok = ok && mbar_wait(bar(B_P_EMPTY + (gv - 2) % kPTiles), ((gv - 2) / kPTiles) & 1, wc, 4);
+          const uint32_t vs = gv % C::NSTG;
+          // the stage's previous tile was read by the PV of step gv - NSTG
+          if (gv >= (uint32_t)C::NSTG) ok = ok && mbar_wait(bar(B_V_EMPTY + vs), ((gv / C::NSTG) - 1) & 1, wc, 4);
           if (ok) {
             const int16_t* my_list = lists + (2 * x + slot) * kMaxBlocks;
             const int kvr = kvrow.get(x);
@@ -408,14 +406,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               for (int hh = 0; hh < C::DH; ++hh)
                 tma_load_2d(dv + hh * C::KVAtom + bb * BS * 128, &tmV, 64 * hh, row, bar(B_V_FULL + vs));
             }
-            lastV = (lastV & ~(5u << vs)) | (1u << vs) | (((gv >> 1) & 1u) << (2 + vs));
+            lastV = (lastV & ~(0x101u << vs)) | (1u << vs) | (((gv / C::NSTG) & 1u) << (8 + vs));
           }
           ++gv;
           if (c == wk.C.get(x) - 1) mbar_arrive(bar(B_ITEM_EMPTY + 2 * x + slot));
           wk.advance(x);
         }
-        for (int u = 0; u < 2; ++u)
-          if (lastV & (1u << u)) mbar_drain(bar(B_V_FULL + u), (lastV >> (2 + u)) & 1u, a.hdr, kKernAttnTc, 5);
+        for (int u = 0; u < C::NSTG; ++u)
+          if (lastV & (1u << u)) mbar_drain(bar(B_V_FULL + u), (lastV >> (8 + u)) & 1u, a.hdr, kKernAttnTc, 5);
       }
     } else if (warp == 1 || warp == 2) {
       // ---------------------------------------------------------------- MMA issuers
@@ -435,8 +433,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         uint32_t n = 0;
         for (;; ++n) {
           if (is_s) {
-            const uint32_t ks = n & 1;
-            const int w = step_wait(bar(B_K_FULL + ks), (n >> 1) & 1, sTotal, n, wc, 14);
+            const uint32_t ks = n % C::NSTG;
+            const int w = step_wait(bar(B_K_FULL + ks), (n / C::NSTG) & 1, sTotal, n, wc, 14);
             if (w <= 0) break;
             const uint32_t meta = sKMeta[ks];
             const int x = (int)(meta & 1u);
@@ -456,18 +454,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                        kk > 0 ? 1u : 0u);
             }
             sStep[2 * x + sb] = n;
-            tc_commit(bar(B_S_FULL + 2 * x + sb));  // also frees K stage ks
+            tc_commit(bar(B_S_FULL + 2 * x + sb));
+            tc_commit(bar(B_K_EMPTY + ks));           // K stage ks may be refilled
             mbar_arrive(bar(B_S_FULL + 2 * x + sb));  // releases the step id
             if (meta & 4u) tc_commit(bar(B_Q_EMPTY + x));
             gs.inc(x);
           } else {
-            const uint32_t vs = n & 1;
-            const uint32_t pt = n % kPTiles, pu = n / kPTiles;
+            const uint32_t vs = n % C::NSTG;
+            const uint32_t pt = n % C::PT, pu = n / C::PT;
             const int w = step_wait(bar(B_P_FULL + pt), pu & 1, sTotal, n, wc, 10);
             if (w <= 0) break;
             const uint32_t meta = sPMeta[pt];
             const int x = (int)(meta & 1u);
-            ok = ok && mbar_wait(bar(B_V_FULL + vs), (n >> 1) & 1, wc, 11);
+            ok = ok && mbar_wait(bar(B_V_FULL + vs), (n / C::NSTG) & 1, wc, 11);
             tc_fence_after();
             if (ok) {
               // only the chunk's kept blocks enter: the rest of the stage is stale
@@ -488,14 +487,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                          kk > 0 ? 1u : acc0);
               }
             }
-            tc_commit(bar(B_P_EMPTY + pt));  // frees P tile pt and V stage vs
+            tc_commit(bar(B_P_EMPTY + pt));  // P tile pt may be rewritten
+            tc_commit(bar(B_V_EMPTY + vs));  // V stage vs may be refilled
             if (meta & 4u) tc_commit(bar(B_O_DONE + x));
           }
         }
         const uint32_t gv = n;
         // the tensor core has finished every MMA before TMEM is released
         if (!is_s && gv > 0)
-          mbar_drain(bar(B_P_EMPTY + (gv - 1) % kPTiles), ((gv - 1) / kPTiles) & 1, a.hdr, kKernAttnTc, 16);
+          mbar_drain(bar(B_P_EMPTY + (gv - 1) % C::PT), ((gv - 1) / C::PT) & 1, a.hdr, kKernAttnTc, 16);
         for (int x = 0; x < kStreams; ++x) {
           const uint32_t ns = gs.get(x);
           if (is_s && ns > 0)
@@ -526,7 +526,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     uint32_t lastn = 0;   // walk step of this stream's previous tile
     // wait until the PV of walk step n has finished
     auto wait_step_pv = [&](uint32_t n) {
-      mbar_wait<true>(bar(B_P_EMPTY + n % kPTiles), (n / kPTiles) & 1, wc, 20);
+      mbar_wait<true>(bar(B_P_EMPTY + n % C::PT), (n / C::PT) & 1, wc, 20);
     };
     for (int t = 0;; ++t) {
       const int slot = t & 1;
@@ -641,9 +641,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mbar_arrive(bar(B_S_FREE + 2 * x + sb));  // the S^T buffer may be refilled
         ++gs;
         // P = 2^(S * scale - m) in bf16, row r of the MN-major P^T tile; the row
-        // sums add the same bf16 values. The tile was last read by step n - kPTiles.
-        if (n_step >= (uint32_t)kPTiles) wait_step_pv(n_step - kPTiles);
-        uint8_t* const prow = smem + C::OffP + (n_step % kPTiles) * C::PBytes + r * C::PRow;
+        // sums add the same bf16 values. The tile was last read by step n - PT.
+        if (n_step >= (uint32_t)C::PT) wait_step_pv(n_step - C::PT);
+        uint8_t* const prow = smem + C::OffP + (n_step % C::PT) * C::PBytes + r * C::PRow;
         // 16-byte chunk cc of this key row sits at chunk cc ^ (row bits of the swizzle)
         const int swz = BS == 64 ? (r & 7) : ((r >> 1) & 3);
         if (!valid) {
@@ -681,10 +681,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             *reinterpret_cast<uint4*>(prow + ((cc ^ swz) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
-        if (r == 0) sPMeta[n_step % kPTiles] = step_meta(x, c == 0, c == Cn - 1, nblk);
+        if (r == 0) sPMeta[n_step % C::PT] = step_meta(x, c == 0, c == Cn - 1, nblk);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
-        mbar_arrive(bar(B_P_FULL + n_step % kPTiles));
+        mbar_arrive(bar(B_P_FULL + n_step % C::PT));
         lastn = n_step;
       }
       // ---------------------------------------------------------------- epilogue

@@ -63,10 +63,13 @@ def _attention_chunk(items: List[Item], block: int, scale: float):
                               items=items)
 
 
-def _backward_chunk(items: List[Item], block: int, scale: float):
+def _backward_chunk(items: List[Item], block: int, scale: float, keep_dq=None):
     from . import dsa_oracle as o
-    return o.sparse_attention_backward(_get("q"), _get("k"), _get("v"), _get("dout"), _get("idx"),
-                                       _get("cnt"), block, scale, items=items)
+    dq, dk, dv = o.sparse_attention_backward(_get("q"), _get("k"), _get("v"), _get("dout"), _get("idx"),
+                                             _get("cnt"), block, scale, items=items)
+    if keep_dq is not None:
+        dq = {it: val for it, val in dq.items() if it in keep_dq}
+    return dq, dk, dv
 
 
 def _select_group(b: int, g: int, group: int, block: int, k_free, local_window: int, n_sink: int,
@@ -127,9 +130,9 @@ class OraclePool:
         self.ex.shutdown(wait=True, cancel_futures=True)
         shutil.rmtree(self.folder, ignore_errors=True)
 
-    def _run(self, fn, items: Iterable[Item], block: int, scale: float, per_worker: int = 4):
+    def _run(self, fn, items: Iterable[Item], block: int, scale: float, per_worker: int = 4, *extra):
         parts = _chunks(list(items), self.workers * per_worker)
-        futs = [self.ex.submit(fn, p, block, scale) for p in parts]
+        futs = [self.ex.submit(fn, p, block, scale, *extra) for p in parts]
         return [f.result() for f in futs]
 
     def attention(self, items: Iterable[Item], block: int, scale: float = 0.0):
@@ -138,9 +141,14 @@ class OraclePool:
             out.update(r)
         return out
 
-    def backward(self, items: Iterable[Item], block: int, scale: float = 0.0):
+    def backward(self, items: Iterable[Item], block: int, scale: float = 0.0, keep_dq=None,
+                 per_worker: int = 4):
+        """The oracle's backward over ``items``; with ``keep_dq`` (a set of
+        items) only those items' dQ blocks are returned (dK, dV always sum
+        every listed item's contribution)."""
         dq, dk, dv = {}, {}, {}
-        for rq, rk, rv in self._run(_backward_chunk, items, block, scale):
+        keep = None if keep_dq is None else set(keep_dq)
+        for rq, rk, rv in self._run(_backward_chunk, items, block, scale, per_worker, keep):
             dq.update(rq)
             for key, val in rk.items():
                 dk[key] = dk[key] + val if key in dk else val

@@ -127,38 +127,3 @@ def test_backward_is_deterministic():
     b = gpu_backward(w, x, do_bits, idx, cnt)
     for ta, tb in zip(a, b):
         assert torch.equal(ta, tb)
-
-
-def test_backward_full_size_32k_sampled():
-    # the benchmark's workload: every gradient tensor checked on sampled blocks
-    w = WORKLOADS["32k-gqa"]
-    x = W.make_inputs(w, seed=68)
-    do_bits = W.f32_to_bf16_bits(np.random.default_rng(69).standard_normal(x["q"].shape).astype(np.float32))
-    idx, cnt = oracle_lists(w, x)
-    dq, dk, dv = gpu_backward(w, x, do_bits, idx, cnt)
-    bs, g = w.block, w.Hq // w.Hkv
-    q_items = [(0, 0, w.nb - 1), (0, 13, 257), (0, 31, 3)]
-    kv_blocks = [(0, 0, w.nb - 1), (0, 5, w.nb - 6), (0, 7, w.nb - 11)]
-    items = set(q_items)
-    for (b, kvh, j) in kv_blocks:
-        for h in range(kvh * g, (kvh + 1) * g):
-            for i in range(j, w.nb):
-                if j in idx[b, h, i, :cnt[b, h, i]]:
-                    items.add((b, h, i))
-    rq, rk, rv = oracle.sparse_attention_backward(x["q"], x["k"], x["v"], do_bits, idx, cnt, bs,
-                                                  items=sorted(items))
-    for (b, h, i) in q_items:
-        check_grad(f"dq{(b, h, i)}", bf16_to_f64(dq[b, h, i * bs:(i + 1) * bs]), rq[(b, h, i)])
-    for (b, kvh, j) in kv_blocks:
-        check_grad(f"dk{(b, kvh, j)}", bf16_to_f64(dk[b, kvh, j * bs:(j + 1) * bs]), rk[(b, kvh, j)])
-        check_grad(f"dv{(b, kvh, j)}", bf16_to_f64(dv[b, kvh, j * bs:(j + 1) * bs]), rv[(b, kvh, j)])
-    # a key block that no list keeps gets exactly zero
-    kept = np.zeros((w.Hkv, w.nb), dtype=bool)
-    for h in range(w.Hq):
-        for i in range(w.nb):
-            kept[h // g, idx[0, h, i, :cnt[0, h, i]]] = True
-    free = np.argwhere(~kept)
-    if free.size:
-        kvh, j = free[0]
-        assert torch.count_nonzero(dk[0, kvh, j * bs:(j + 1) * bs]) == 0
-        assert torch.count_nonzero(dv[0, kvh, j * bs:(j + 1) * bs]) == 0

@@ -1,9 +1,8 @@
 """GPU parity: every step of the CUDA path against the fp64 oracle, through the C ABI.
 
 Small cases span several tiles and ragged tails (nb not a multiple of the
-32-lane selection warp, odd block counts, per-head budgets, empty rows); the
-full-size workloads are checked in the launch configuration the benchmark
-uses, on the whole selection and on sampled query blocks of the attention.
+32-lane selection warp, odd block counts, per-head budgets, empty rows). The
+full-size workloads are checked in tests/test_gpu_fullsize.py.
 """
 import numpy as np
 import pytest
@@ -200,55 +199,3 @@ def test_cuda_graph_capture_replays_forward():
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
-
-
-# ---------------------------------------------------------------------------
-# Full-size workloads, in the benchmark's launch configuration (dsa_forward).
-# ---------------------------------------------------------------------------
-
-def sample_items(w, n, seed):
-    g = np.random.default_rng(seed)
-    items = {(int(g.integers(w.B)), int(g.integers(w.Hq)), int(g.integers(w.nb))) for _ in range(n)}
-    for h in range(0, w.Hq, max(1, w.Hq // 4)):
-        items.add((w.B - 1, h, w.nb - 1))
-        items.add((0, h, 0))
-    return sorted(items)
-
-
-@pytest.mark.parametrize("name", ["tiny", "8k-gqa", "32k-gqa", "128k-structured", "batched-32"])
-def test_full_workload(name):
-    w = WORKLOADS[name]
-    kph = W.per_head_k(w)
-    kph_l = None if kph is None else [int(t) for t in kph]
-    x = W.make_inputs(w)
-    s64, idx_ref, cnt_ref = oracle_reference(w, x, kph_l)
-
-    q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
-    att = BlockSparseAttention.from_workload(w, k_per_head=kph_l)
-    idx_g, cnt_g = att.empty_selection()
-    out, lse = att.empty_out(), att.empty_lse()
-    att.forward(q, k, v, out, lse, idx_g, cnt_g)
-    assert att.check_status() == B.DSA_OK
-    idx_h, cnt_h = idx_g.cpu().numpy(), cnt_g.cpu().numpy()
-    n, ties, bad = compare_selection(idx_h, cnt_h, idx_ref, cnt_ref, s64, per_head(w, kph_l),
-                                     w.local_window, w.n_sink)
-    print(f"{name}: {n} rows, {ties} near-tie rows, {len(bad)} mismatches")
-    assert not bad, bad[:5]
-
-    items = sample_items(w, 24 if w.N >= 32768 else 64, seed=11)
-    ref = oracle.sparse_attention(x["q"], x["k"], x["v"], idx_ref, cnt_ref, w.block, items=items)
-    out2, lse2 = att.empty_out(), att.empty_lse()
-    att.sparse_attn(q, k, v, dev_i32(idx_ref), dev_i32(cnt_ref), out2, lse2)
-    assert att.check_status() == B.DSA_OK
-    bs = w.block
-    o_g = np.concatenate([out2[b, h, i * bs:(i + 1) * bs].double().cpu().numpy() for (b, h, i) in items])
-    o_r = np.concatenate([ref[it][0] for it in items])
-    assert_attention_close(o_g, o_r, name)
-    l_g = np.concatenate([lse2[b, h, i * bs:(i + 1) * bs].double().cpu().numpy() for (b, h, i) in items])
-    l_r = np.concatenate([ref[it][1] for it in items])
-    assert_lse_close(l_g, l_r, name)
-    # dsa_forward's own output on sampled blocks whose selection equals the oracle's
-    keep = [it for it in items if np.array_equal(idx_h[it], idx_ref[it])]
-    o_f = np.concatenate([out[b, h, i * bs:(i + 1) * bs].double().cpu().numpy() for (b, h, i) in keep])
-    o_r2 = np.concatenate([ref[it][0] for it in keep])
-    assert_attention_close(o_f, o_r2, name + " fused")
