@@ -484,7 +484,7 @@ __global__ void __launch_bounds__(BwdCfg<BS, D>::kThreads) bwd_dkv_kernel(BwdArg
 }
 
 template <int BS, int D>
-cudaError_t launch_bwd_impl(const BwdArgs& a, cudaStream_t st) {
+cudaError_t launch_bwd_impl(const BwdArgs& a, const Shape& s, const BwdTcArgs* tc, cudaStream_t st) {
   using Cfg = BwdCfg<BS, D>;
   cudaError_t e;
   {
@@ -505,6 +505,8 @@ cudaError_t launch_bwd_impl(const BwdArgs& a, cudaStream_t st) {
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
   }
+  // the tensor-core passes (attn_bwd_tc.cu) take over from here
+  if (tc != nullptr) return launch_attn_bwd_tc(s, *tc, st);
   {
     auto f = bwd_dq_kernel<BS, D>;
     e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::kSmemDq);
@@ -532,7 +534,7 @@ cudaError_t launch_attn_bwd(const Shape& s, const __nv_bfloat16* q, const __nv_b
                             const __nv_bfloat16* v, const __nv_bfloat16* o, const float* lse,
                             const __nv_bfloat16* dout, const int32_t* idx, const int32_t* cnt,
                             __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, void* ws,
-                            cudaStream_t st) {
+                            bool use_tc, cudaStream_t st) {
   const BwdWs lw = bwd_ws_layout(s);
   char* base = static_cast<char*>(ws);
   BwdArgs a;
@@ -561,12 +563,42 @@ cudaError_t launch_attn_bwd(const Shape& s, const __nv_bfloat16* q, const __nv_b
   a.cw = lw.cw;
   a.scale = s.scale;
   a.c2 = s.scale * kLog2e;
-  if (s.bs == 32 && s.d == 64) return launch_bwd_impl<32, 64>(a, st);
-  if (s.bs == 64 && s.d == 64) return launch_bwd_impl<64, 64>(a, st);
-  if (s.bs == 128 && s.d == 64) return launch_bwd_impl<128, 64>(a, st);
-  if (s.bs == 32 && s.d == 128) return launch_bwd_impl<32, 128>(a, st);
-  if (s.bs == 64 && s.d == 128) return launch_bwd_impl<64, 128>(a, st);
-  if (s.bs == 128 && s.d == 128) return launch_bwd_impl<128, 128>(a, st);
+  BwdTcArgs t;
+  const BwdTcArgs* tc = nullptr;
+  if (use_tc) {
+    t.q = q;
+    t.k = k;
+    t.v = v;
+    t.dout = dout;
+    t.idx = idx;
+    t.cnt = cnt;
+    t.drow = a.drow;
+    t.lse2 = a.lse2;
+    t.colbits = a.colbits;
+    t.pairs = reinterpret_cast<int32_t*>(base + lw.pairs);
+    t.npairs = reinterpret_cast<int32_t*>(base + lw.npairs);
+    t.dq = dq;
+    t.dk = dk;
+    t.dv = dv;
+    t.hdr = a.hdr;
+    t.B = s.B;
+    t.Hq = s.Hq;
+    t.Hkv = s.Hkv;
+    t.N = s.N;
+    t.nb = s.nb;
+    t.W = s.W;
+    t.group = s.group;
+    t.cw = lw.cw;
+    t.scale = s.scale;
+    t.c2 = a.c2;
+    tc = &t;
+  }
+  if (s.bs == 32 && s.d == 64) return launch_bwd_impl<32, 64>(a, s, tc, st);
+  if (s.bs == 64 && s.d == 64) return launch_bwd_impl<64, 64>(a, s, tc, st);
+  if (s.bs == 128 && s.d == 64) return launch_bwd_impl<128, 64>(a, s, tc, st);
+  if (s.bs == 32 && s.d == 128) return launch_bwd_impl<32, 128>(a, s, tc, st);
+  if (s.bs == 64 && s.d == 128) return launch_bwd_impl<64, 128>(a, s, tc, st);
+  if (s.bs == 128 && s.d == 128) return launch_bwd_impl<128, 128>(a, s, tc, st);
   return cudaErrorInvalidValue;
 }
 

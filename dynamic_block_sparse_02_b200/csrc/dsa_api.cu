@@ -397,11 +397,14 @@ dsa_status dsa_sparse_attn_bwd(const dsa_params* p, const dsa_bf16* q, const dsa
     return DSA_ERR_INVALID_ARG;
   if (ws == nullptr || !aligned16(ws) || ws_bytes < dsa::bwd_ws_layout(s).total) return DSA_ERR_WORKSPACE;
   if ((st = check_device()) != DSA_OK) return st;
+  const bool tc_ok = dsa::attn_bwd_tc_supported(s);
+  if (p->attn_kernel == DSA_ATTN_TCGEN05 && !tc_ok) return DSA_ERR_UNSUPPORTED;
+  const bool use_tc = tc_ok && p->attn_kernel != DSA_ATTN_MMA_SYNC;
   return from_cuda(dsa::launch_attn_bwd(
       s, reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k),
       reinterpret_cast<const __nv_bfloat16*>(v), reinterpret_cast<const __nv_bfloat16*>(out), lse,
       reinterpret_cast<const __nv_bfloat16*>(dout), idx, cnt, reinterpret_cast<__nv_bfloat16*>(dq),
-      reinterpret_cast<__nv_bfloat16*>(dk), reinterpret_cast<__nv_bfloat16*>(dv), ws,
+      reinterpret_cast<__nv_bfloat16*>(dk), reinterpret_cast<__nv_bfloat16*>(dv), ws, use_tc,
       (cudaStream_t)stream));
 }
 

@@ -96,8 +96,11 @@ inline DecodeWs decode_ws_layout(const Shape& s) {
 // Backward workspace after the header: fp32 D_r = dO_r . O_r and base-2 lse
 // per query row [B, Hq, N], and the transposed kept lists, one bitmap of
 // cw = ceil(G * nb / 32) words per key block [B, Hkv, nb, cw].
+// For the tensor-core backward also the transposed lists as pair lists
+// (int32 bit positions, G (nb - j) slots for key block j, packed per (b, g):
+// [B, Hkv, G nb (nb + 1) / 2]) and their lengths [B, Hkv, nb].
 struct BwdWs {
-  size_t drow, lse2, colbits, total;
+  size_t drow, lse2, colbits, pairs, npairs, total;
   int cw;
 };
 inline BwdWs bwd_ws_layout(const Shape& s) {
@@ -110,16 +113,44 @@ inline BwdWs bwd_ws_layout(const Shape& s) {
   off += ws_round_up((size_t)s.B * s.Hq * s.N * sizeof(float));
   w.colbits = off;
   off += ws_round_up((size_t)s.B * s.Hkv * s.nb * w.cw * sizeof(uint32_t));
+  w.pairs = off;
+  off += ws_round_up((size_t)s.B * s.Hkv * s.group * ((size_t)s.nb * (s.nb + 1) / 2) * sizeof(int32_t));
+  w.npairs = off;
+  off += ws_round_up((size_t)s.B * s.Hkv * s.nb * sizeof(int32_t));
   w.total = off;
   return w;
 }
+
+// Arguments of the tensor-core backward (attn_bwd_tc.cu).
+struct BwdTcArgs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const __nv_bfloat16* dout;
+  const int32_t* idx;
+  const int32_t* cnt;
+  const float* drow;   // D_r = dO_r . O_r
+  const float* lse2;   // lse * log2(e), +inf for a row with no visible key
+  const uint32_t* colbits;
+  int32_t* pairs;
+  int32_t* npairs;
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  WsHeader* hdr;
+  int B, Hq, Hkv, N, nb, W, group, cw;
+  float scale, c2;
+};
+bool attn_bwd_tc_supported(const Shape& s);
+// dQ, dK, dV on the tensor cores, after the D / lse2 and bitmap kernels.
+cudaError_t launch_attn_bwd_tc(const Shape& s, const BwdTcArgs& a, cudaStream_t st);
 
 // Backward of the sparse attention over the kept blocks (dQ, dK, dV).
 cudaError_t launch_attn_bwd(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
                             const __nv_bfloat16* v, const __nv_bfloat16* o, const float* lse,
                             const __nv_bfloat16* dout, const int32_t* idx, const int32_t* cnt,
                             __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, void* ws,
-                            cudaStream_t st);
+                            bool use_tc, cudaStream_t st);
 
 // Decode step: one query token per (batch, query head) at position length - 1.
 cudaError_t launch_decode(const Shape& s, const KBudget& kb, const __nv_bfloat16* q,

@@ -68,8 +68,11 @@ def test_kmax_and_workspace_size(name):
     # decode: scores [B, Hq, nb], partial states [B, Hq, min(64, nb), d + 4], counters
     decode = 256 + rnd(w.B * w.Hq * w.nb * 4) + rnd(w.B * w.Hq * min(64, w.nb) * (w.d + 4) * 4) \
         + rnd(w.B * w.Hkv * -(-(w.Hq // w.Hkv) // 8) * 4)
-    # backward: D and base-2 lse per query row, one bitmap of ceil(G * nb / 32) words per key block
-    backward = 256 + 2 * rnd(w.B * w.Hq * w.N * 4) + rnd(w.B * w.Hkv * w.nb * -(-(w.Hq // w.Hkv * w.nb) // 32) * 4)
+    # backward: D and base-2 lse per query row, one bitmap of ceil(G * nb / 32) words per key block,
+    # the pair lists (G (nb - j) int32 slots for key block j) and their lengths
+    G = w.Hq // w.Hkv
+    backward = 256 + 2 * rnd(w.B * w.Hq * w.N * 4) + rnd(w.B * w.Hkv * w.nb * -(-(G * w.nb) // 32) * 4) \
+        + rnd(w.B * w.Hkv * G * (w.nb * (w.nb + 1) // 2) * 4) + rnd(w.B * w.Hkv * w.nb * 4)
     assert ws == max(prefill, decode, backward)
 
 

@@ -39,8 +39,11 @@ def oracle_lists(w, x):
     return oracle.select_blocks(s, w.k_free, w.local_window, w.n_sink)
 
 
-def gpu_backward(w, x, do_bits, idx, cnt):
-    att = BlockSparseAttention.from_workload(w)
+KERNELS = [B.DSA_ATTN_AUTO, B.DSA_ATTN_MMA_SYNC]
+
+
+def gpu_backward(w, x, do_bits, idx, cnt, kernel=B.DSA_ATTN_AUTO):
+    att = BlockSparseAttention.from_workload(w, attn_kernel=kernel)
     q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
     di, dc = dev_i32(idx), dev_i32(cnt)
     out = torch.empty_like(q)
@@ -73,21 +76,23 @@ CASES = {
 }
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("name", list(CASES))
-def test_backward_parity(name):
+def test_backward_parity(name, kernel):
     Bn, Hq, Hkv, N, d, bs, k, lw, ns = CASES[name]
     w = Workload(name, Bn, Hq, Hkv, N, d, bs, k_free=k, local_window=lw, n_sink=ns)
     x = W.make_inputs(w, seed=61)
     do_bits = W.f32_to_bf16_bits(np.random.default_rng(62).standard_normal(x["q"].shape).astype(np.float32))
     idx, cnt = oracle_lists(w, x)
-    dq, dk, dv = gpu_backward(w, x, do_bits, idx, cnt)
+    dq, dk, dv = gpu_backward(w, x, do_bits, idx, cnt, kernel)
     rq, rk, rv = oracle.sparse_attention_backward(x["q"], x["k"], x["v"], do_bits, idx, cnt, bs)
     check_grad("dq", bf16_to_f64(dq), rq)
     check_grad("dk", bf16_to_f64(dk), rk)
     check_grad("dv", bf16_to_f64(dv), rv)
 
 
-def test_backward_caller_lists_with_empty_rows_and_no_diagonal():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_backward_caller_lists_with_empty_rows_and_no_diagonal(kernel):
     # rows with no kept block (lse = -inf: no gradient) and rows whose list
     # skips the diagonal block
     w = Workload("custom", 1, 4, 2, 64 * 8, 128, 64, k_free=3, local_window=1, n_sink=0)
@@ -105,7 +110,7 @@ def test_backward_caller_lists_with_empty_rows_and_no_diagonal():
             lst = sorted(rng.choice(pool, size=min(width, len(pool)), replace=False).tolist())
             idx[0, h, i, :len(lst)] = lst
             cnt[0, h, i] = len(lst)
-    dq, dk, dv = gpu_backward(w, x, do_bits, idx, cnt)
+    dq, dk, dv = gpu_backward(w, x, do_bits, idx, cnt, kernel)
     rq, rk, rv = oracle.sparse_attention_backward(x["q"], x["k"], x["v"], do_bits, idx, cnt, w.block)
     check_grad("dq", bf16_to_f64(dq), rq)
     check_grad("dk", bf16_to_f64(dk), rk)
@@ -117,13 +122,14 @@ def test_backward_caller_lists_with_empty_rows_and_no_diagonal():
                 assert np.all(gq[0, h, i * 64:(i + 1) * 64] == 0)
 
 
-def test_backward_is_deterministic():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_backward_is_deterministic(kernel):
     Bn, Hq, Hkv, N, d, bs, k, lw, ns = CASES["gqa-d128-bs64"]
     w = Workload("det", Bn, Hq, Hkv, N, d, bs, k_free=k, local_window=lw, n_sink=ns)
     x = W.make_inputs(w, seed=66)
     do_bits = W.f32_to_bf16_bits(np.random.default_rng(67).standard_normal(x["q"].shape).astype(np.float32))
     idx, cnt = oracle_lists(w, x)
-    a = gpu_backward(w, x, do_bits, idx, cnt)
-    b = gpu_backward(w, x, do_bits, idx, cnt)
+    a = gpu_backward(w, x, do_bits, idx, cnt, kernel)
+    b = gpu_backward(w, x, do_bits, idx, cnt, kernel)
     for ta, tb in zip(a, b):
         assert torch.equal(ta, tb)
