@@ -125,5 +125,9 @@ class BlockSparseAttention:
                          self.ws, self.ws_bytes, self.stream)
         return out
 
+    def set_wait_limit(self, ns: int) -> None:
+        """Time limit (ns) of the kernels' bounded waits; 0 = the default."""
+        B.dsa_workspace_set_wait_limit(self.ws, self.ws_bytes, ns, self.stream)
+
     def check_status(self) -> int:
         return B.dsa_check_status(self.ws, self.stream)

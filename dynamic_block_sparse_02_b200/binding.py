@@ -57,6 +57,7 @@ SIGNATURES = {
     "dsa_kmax": (_sz, [_P]),
     "dsa_workspace_size": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_size_t)]),
     "dsa_workspace_init": (ctypes.c_int, [_vp, _sz, _vp]),
+    "dsa_workspace_set_wait_limit": (ctypes.c_int, [_vp, _sz, ctypes.c_ulonglong, _vp]),
     "dsa_block_scores": (ctypes.c_int, [_P, _vp, _vp, _f32p, _vp, _sz, _vp]),
     "dsa_topk_select": (ctypes.c_int, [_P, _f32p, _i32p, _i32p, _vp]),
     "dsa_select_blocks": (ctypes.c_int, [_P, _vp, _vp, _i32p, _i32p, _vp, _sz, _vp]),
@@ -162,6 +163,11 @@ def dsa_workspace_size(p: Params) -> int:
 
 def dsa_workspace_init(ws, ws_bytes: int, stream=None) -> None:
     _check(_lib.dsa_workspace_init(_ptr(ws), ws_bytes, _stream(stream)), "dsa_workspace_init")
+
+
+def dsa_workspace_set_wait_limit(ws, ws_bytes: int, ns: int, stream=None) -> None:
+    _check(_lib.dsa_workspace_set_wait_limit(_ptr(ws), ws_bytes, int(ns), _stream(stream)),
+           "dsa_workspace_set_wait_limit")
 
 
 def dsa_block_scores(p: Params, q, k, scores, ws, ws_bytes: int, stream=None) -> None:

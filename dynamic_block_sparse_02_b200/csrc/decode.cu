@@ -246,17 +246,12 @@ __host__ __device__ inline AttnSmem attn_smem(int D, int nb, int W, int bs, int 
 
 constexpr unsigned long long kDecWaitLimitNs = 1000000000ull;  // 1 s
 
-__device__ __forceinline__ unsigned long long dec_now_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ bool dbar_try(uint32_t bar, uint32_t parity) {
+// Non-suspending test of a phase.
+__device__ __forceinline__ bool dbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -264,28 +259,37 @@ __device__ __forceinline__ bool dbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for a phase of a stage barrier: false (with the CTA abort flag
-// and the device error raised) when it does not complete within the limit, or
-// at once when the CTA is already aborting (abort_flag may be null).
+// A wait with an abort flag uses the workspace header's limit when one is set
+// (WsHeader::wait_limit_ns, so that a test can make it give up); the drain
+// after an abort (abort_flag null) always allows the default limit. The spin
+// polls without suspending and measures SM cycles (fine-grained, unlike the
+// global timer), counting 2 cycles per ns: the limit holds at clocks up to
+// 2 GHz and is longer below.
 __device__ __noinline__ bool dbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                             WsHeader* hdr, int where) {
-  const unsigned long long t0 = dec_now_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (dbar_try(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
-      if (abort_flag != nullptr && *abort_flag) return false;
-      if (dec_now_ns() - t0 > kDecWaitLimitNs) {
-        if (abort_flag != nullptr) *abort_flag = 1;
-        raise_error(hdr, DSA_ERR_DEVICE_TIMEOUT, kKernDecode, where, (int)blockIdx.x);
-        return false;
-      }
+  const long long c0 = clock64();
+  unsigned long long limit = kDecWaitLimitNs;
+  if (abort_flag != nullptr && hdr != nullptr) {
+    const unsigned long long v = *reinterpret_cast<const volatile unsigned long long*>(&hdr->wait_limit_ns);
+    if (v != 0ull) limit = v;
+  }
+  const long long lim_cycles = (long long)(limit < 4000000000ull ? limit : 4000000000ull) * 2;
+  for (;;) {
+    if (dbar_test(bar, parity)) return true;
+    if (abort_flag != nullptr && *abort_flag) return false;
+    if (clock64() - c0 > lim_cycles) {
+      if (abort_flag != nullptr) *abort_flag = 1;
+      raise_error(hdr, DSA_ERR_DEVICE_TIMEOUT, kKernDecode, where, (int)blockIdx.x);
+      return false;
     }
   }
 }
 
+// The first probe does not suspend, so a stage that has not arrived always
+// reaches the bounded spin (and its time limit).
 __device__ __forceinline__ bool dbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           WsHeader* hdr, int where) {
-  if (dbar_try(bar, parity)) return true;
+  if (dbar_test(bar, parity)) return true;
   return dbar_wait_slow(bar, parity, abort_flag, hdr, where);
 }
 

@@ -260,6 +260,9 @@ size_t static_scratch_need(const Shape& s, size_t* kp_off) {
   return *kp_off + round_up((size_t)s.B * s.Hkv * s.nb * s.d * sizeof(float));
 }
 
+// Writes the wait limit into a workspace header (one thread).
+__global__ void set_wait_limit_kernel(dsa::WsHeader* hdr, unsigned long long ns) { hdr->wait_limit_ns = ns; }
+
 }  // namespace
 
 extern "C" {
@@ -288,6 +291,13 @@ dsa_status dsa_workspace_size(const dsa_params* p, size_t* bytes) {
 dsa_status dsa_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (ws == nullptr || !aligned16(ws) || ws_bytes < dsa::kHeaderBytes) return DSA_ERR_WORKSPACE;
   return from_cuda(cudaMemsetAsync(ws, 0, dsa::kHeaderBytes, (cudaStream_t)stream));
+}
+
+dsa_status dsa_workspace_set_wait_limit(void* ws, size_t ws_bytes, unsigned long long ns, void* stream) {
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < dsa::kHeaderBytes) return DSA_ERR_WORKSPACE;
+  if (check_device() != DSA_OK) return DSA_ERR_UNSUPPORTED;
+  set_wait_limit_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(static_cast<dsa::WsHeader*>(ws), ns);
+  return from_cuda(cudaGetLastError());
 }
 
 dsa_status dsa_block_scores(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k,

@@ -69,7 +69,9 @@ struct WaitCtx {
 // Bounded wait. Returns false (and raises the CTA abort flag and the device
 // error) when the phase does not complete within the limit, or at once when
 // the CTA is already aborting. The first probe is inlined; the spin loop is
-// out of line so that callers keep their registers on the fast path.
+// out of line so that callers keep their registers on the fast path. A
+// try_wait may itself suspend for a while, so the limit and the abort flag are
+// checked after the first failed probe and then every 8 probes.
 template <bool kInline>
 __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, volatile CtaFlags* f,
                                                WsHeader* hdr, int kernel, int where) {
@@ -77,7 +79,7 @@ __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, vo
   const unsigned long long limit = f->limit_ns;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
+    if (it == 1u || (it & 7u) == 0u) {
       if (f->abort) return false;
       if (now_ns() - t0 > limit) {
         f->abort = 1;
@@ -112,7 +114,7 @@ __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, WsHead
   const unsigned long long t0 = now_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
-    if ((it & 63u) == 0u && now_ns() - t0 > kDefaultWaitNs) {
+    if ((it == 1u || (it & 7u) == 0u) && now_ns() - t0 > kDefaultWaitNs) {
       raise_error(hdr, DSA_ERR_DEVICE_TIMEOUT, kernel, where, (int)blockIdx.x);
       return false;
     }
@@ -130,7 +132,7 @@ static __device__ __noinline__ int step_wait_slow(uint32_t bar, uint32_t parity,
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return 1;
     if (*total <= n) return 0;
-    if ((it & 63u) == 0u) {
+    if (it == 1u || (it & 7u) == 0u) {
       if (f->abort) return -1;
       if (now_ns() - t0 > limit) {
         f->abort = 1;

@@ -147,6 +147,21 @@ dsa_status dsa_workspace_size(const dsa_params *p, size_t *bytes);
 dsa_status dsa_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Set the time limit of the kernels' bounded waits for calls that use this
+ * workspace (asynchronous on `stream`; stored in the workspace header, which
+ * dsa_workspace_init resets to 0). ns = 0 selects the default (2 s for the
+ * tensor-core kernels, 1 s for the decode kernel). Every wait inside the
+ * pipelined kernels (a stage that has not arrived, a buffer not yet released)
+ * is bounded: when one gives up, the kernel raises DSA_ERR_DEVICE_TIMEOUT,
+ * stops issuing work, waits (with the default limit) for the copies and
+ * tensor-core products it has in flight, frees its tensor memory and returns;
+ * its outputs are then undefined. A tiny limit makes the waits give up on
+ * purpose, which is how the failure path is tested. There is no counterpart
+ * in the pages: the pages describe no failure handling.
+ */
+dsa_status dsa_workspace_set_wait_limit(void *ws, size_t ws_bytes, unsigned long long ns, void *stream);
+
+/*
  * Steps 1-2. scores: device fp32 [B, Hq, nb, nb]; scores[b,h,i,j] =
  * Qp[b,h,i] . Kp[b,h/(Hq/Hkv),j] for j <= i and -inf for j > i.
  * Uses the workspace for the pooled blocks.
