@@ -363,6 +363,7 @@ def run_ours(args, w):
         dist.barrier()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if needs_flush(w) else None
     torch.cuda.synchronize(dev)
+    torch.cuda.nvtx.range_push("timed steps")
     with torch.cuda.stream(stream):
         for s in range(K):
             if flush is not None:
@@ -373,6 +374,7 @@ def run_ours(args, w):
             attend()
             ev[s][2].record(stream)
     torch.cuda.synchronize(dev)
+    torch.cuda.nvtx.range_pop()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if rank == 0 else None

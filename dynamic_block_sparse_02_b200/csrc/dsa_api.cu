@@ -7,11 +7,21 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "dsa_internal.cuh"
 
 using dsa::Shape;
 
 namespace {
+
+// An NVTX range around one entry point (host side: the range covers the
+// argument checks and the kernel launches, which profilers correlate with the
+// kernels they issued). NVTX costs nothing unless a tool is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 
 constexpr size_t kAlign = 256;
 
@@ -302,6 +312,7 @@ dsa_status dsa_workspace_set_wait_limit(void* ws, size_t ws_bytes, unsigned long
 
 dsa_status dsa_block_scores(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k,
                             float* scores, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("dsa_block_scores");
   Shape s;
   dsa_status st = make_shape(p, &s);
   if (st != DSA_OK) return st;
@@ -324,6 +335,7 @@ dsa_status dsa_block_scores(const dsa_params* p, const dsa_bf16* q, const dsa_bf
 
 dsa_status dsa_topk_select(const dsa_params* p, const float* scores, int32_t* idx, int32_t* cnt,
                            void* stream) {
+  NvtxRange nvtx("dsa_topk_select");
   Shape s;
   dsa_status st = make_shape(p, &s);
   if (st != DSA_OK) return st;
@@ -336,6 +348,7 @@ dsa_status dsa_topk_select(const dsa_params* p, const float* scores, int32_t* id
 
 dsa_status dsa_select_blocks(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k,
                              int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("dsa_select_blocks");
   Shape s;
   dsa_status st = make_shape(p, &s);
   if (st != DSA_OK) return st;
@@ -350,6 +363,7 @@ dsa_status dsa_select_blocks(const dsa_params* p, const dsa_bf16* q, const dsa_b
 
 dsa_status dsa_select_blocks_static(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k,
                                     int32_t* idx, int32_t* cnt, void* stream) {
+  NvtxRange nvtx("dsa_select_blocks_static");
   Shape s;
   dsa_status st = make_shape(p, &s);
   if (st != DSA_OK) return st;
@@ -377,6 +391,7 @@ dsa_status dsa_select_blocks_static(const dsa_params* p, const dsa_bf16* q, cons
 dsa_status dsa_sparse_attn_fwd(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k,
                                const dsa_bf16* v, const int32_t* idx, const int32_t* cnt,
                                dsa_bf16* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("dsa_sparse_attn_fwd");
   Shape s;
   dsa_status st = make_shape(p, &s);
   if (st != DSA_OK) return st;
@@ -396,6 +411,7 @@ dsa_status dsa_sparse_attn_bwd(const dsa_params* p, const dsa_bf16* q, const dsa
                                const dsa_bf16* dout, const int32_t* idx, const int32_t* cnt,
                                dsa_bf16* dq, dsa_bf16* dk, dsa_bf16* dv, void* ws, size_t ws_bytes,
                                void* stream) {
+  NvtxRange nvtx("dsa_sparse_attn_bwd");
   Shape s;
   dsa_status st = make_shape(p, &s);
   if (st != DSA_OK) return st;
@@ -421,6 +437,7 @@ dsa_status dsa_sparse_attn_bwd(const dsa_params* p, const dsa_bf16* q, const dsa
 dsa_status dsa_forward(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k, const dsa_bf16* v,
                        dsa_bf16* out, float* lse, int32_t* idx, int32_t* cnt, void* ws,
                        size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("dsa_forward");
   Shape s;
   dsa_status st = make_shape(p, &s);
   if (st != DSA_OK) return st;
@@ -447,6 +464,7 @@ dsa_status dsa_forward(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k
 
 dsa_status dsa_pool_keys(const dsa_params* p, const dsa_bf16* k, float* kp, int j_begin, int j_end,
                          void* stream) {
+  NvtxRange nvtx("dsa_pool_keys");
   Shape s;
   dsa_status st = make_shape(p, &s);
   if (st != DSA_OK) return st;
@@ -462,6 +480,7 @@ dsa_status dsa_pool_keys(const dsa_params* p, const dsa_bf16* k, float* kp, int 
 dsa_status dsa_decode_fwd(const dsa_params* p, const dsa_bf16* q, const dsa_bf16* k,
                           const dsa_bf16* v, const float* kp, int length, dsa_bf16* out, float* lse,
                           int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("dsa_decode_fwd");
   Shape s;
   dsa_status st = make_shape(p, &s);
   if (st != DSA_OK) return st;
