@@ -572,26 +572,33 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmF1, const __grid_constant__ 
         tmem_ld(tmem + lane_addr + 128 + ua * 64 + col0, dp);
         tc_fence_before();
         mbar_arrive(bar(B_A_FREE + ua));
-        // P and G in bf16, packed in pairs of columns
+        // P and G in bf16, packed in pairs of columns (two-wide fp32 math; a
+        // row outside the chunk's loaded blocks is all zeros, the causal mask
+        // applies in the diagonal block only)
         uint32_t gw[16], pw[16];
+        if (!valid) {
 #pragma unroll
-        for (int k2 = 0; k2 < 16; ++k2) {
-          float pv[2], gv[2];
+          for (int k2 = 0; k2 < 16; ++k2) gw[k2] = pw[k2] = 0u;
+        } else {
+          const float2 c22 = make_float2(c2, c2);
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int k = 2 * k2 + e;
-            const int col = col0 + k;
-            const float L = DKV ? ldr.x : ldc[k].x;
-            const float Dv = DKV ? ldr.y : ldc[k].y;
-            // dQ: row r is key rl of block blk, column col a query; dK/dV: row r is
-            // query rl of its pair, column col a key
-            const bool masked = !valid || (diag && (DKV ? col > rl : rl > col));
-            const float p = masked ? 0.f : ex2(__fmaf_rn(__uint_as_float(s[k]), c2, -L));
-            pv[e] = p;
-            gv[e] = masked ? 0.f : p * (__uint_as_float(dp[k]) - Dv);
+          for (int k2 = 0; k2 < 16; ++k2) {
+            const int k = 2 * k2, col = col0 + k;
+            const float2 nl = DKV ? make_float2(-ldr.x, -ldr.x) : make_float2(-ldc[k].x, -ldc[k + 1].x);
+            const float2 dv2 = DKV ? make_float2(ldr.y, ldr.y) : make_float2(ldc[k].y, ldc[k + 1].y);
+            const float2 x2 = __ffma2_rn(make_float2(__uint_as_float(s[k]), __uint_as_float(s[k + 1])), c22, nl);
+            float p0 = ex2(x2.x), p1 = ex2(x2.y);
+            if (diag) {
+              // dQ: row r is key rl, columns are queries; dK/dV: row r is query
+              // rl, columns are keys
+              if (DKV ? col > rl : rl > col) p0 = 0.f;
+              if (DKV ? col + 1 > rl : rl > col + 1) p1 = 0.f;
+            }
+            const float2 dd = make_float2(__uint_as_float(dp[k]) - dv2.x, __uint_as_float(dp[k + 1]) - dv2.y);
+            const float2 g2 = __fmul2_rn(make_float2(p0, p1), dd);
+            if (DKV) pw[k2] = pack_bf16(p0, p1);
+            gw[k2] = pack_bf16(g2.x, g2.y);
           }
-          if (DKV) pw[k2] = pack_bf16(pv[0], pv[1]);
-          gw[k2] = pack_bf16(gv[0], gv[1]);
         }
         // G: the tile was read by the Acc products of step n - NG
         if (n >= (uint32_t)NG) mbar_wait<true>(bar(B_G_EMPTY + ug), ((n / NG) - 1) & 1, wc, 24);
