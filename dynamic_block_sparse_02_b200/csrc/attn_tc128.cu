@@ -33,8 +33,12 @@
 //   warp 3      V producer
 //   warps 4-11  softmax + epilogue, two warpgroups (query columns 0-63, 64-127)
 //
-// Shared memory: Q 32 KB, K ring 2 x 32 KB, V ring 2 x 32 KB, one P^T tile
-// 32 KB (d = 128). Every mbarrier wait is bounded; on expiry the kernel sets
+// Shared memory (d = 128): Q 32 KB, one ring of three 32 KB stages that K and V
+// tiles share (load 2n is K of step n, load 2n + 1 its V, stage = load mod 3;
+// a stage is refilled after the product that read it commits to the stage's
+// empty barrier), and two P^T tiles of 32 KB, so that the softmax of step n
+// writes its P while the PV product of step n - 1 still reads the other tile.
+// Every mbarrier wait is bounded; on expiry the kernel sets
 // DSA_ERR_DEVICE_TIMEOUT, stops issuing work, drains and returns.
 #include "tc_common.cuh"
 
@@ -57,17 +61,17 @@ struct Cfg128 {
   static constexpr int TileBytes = kBS * D * 2;     // Q, K, V tiles: [DH][128 rows][128 B]
   static constexpr int Atom = kBS * 128;            // one d-atom of a tile
   static constexpr int PBytes = kBS * kBS * 2;      // P^T: [2 query halves][128 keys][128 B]
+  static constexpr int NKV = 3;                     // stages of the shared K/V ring
   static constexpr int OffQ = 0;
-  static constexpr int OffK = OffQ + TileBytes;     // 2 stages
-  static constexpr int OffV = OffK + 2 * TileBytes; // 2 stages
-  static constexpr int OffP = OffV + 2 * TileBytes;
-  static constexpr int OffList = OffP + PBytes;     // [slot][kMaxBlocks] int16
+  static constexpr int OffKV = OffQ + TileBytes;    // NKV stages
+  static constexpr int OffP = OffKV + NKV * TileBytes;  // 2 tiles
+  static constexpr int OffList = OffP + 2 * PBytes; // [slot][kMaxBlocks] int16
   static constexpr int OffRed = OffList + 2 * kMaxBlocks * 2;  // [wg][4][64] f32
   static constexpr int OffM = OffRed + 2 * 4 * 64 * 4;         // [wg][64] -(running max)
   static constexpr int OffL = OffM + 2 * 64 * 4;               // [wg][64] 1 / row sum
   static constexpr int OffA = OffL + 2 * 64 * 4;               // [wg][64] max increments
   static constexpr int OffBar = OffA + 2 * 64 * 4;
-  static constexpr int NumBars = 24;
+  static constexpr int NumBars = 28;
   static constexpr int OffMisc = OffBar + NumBars * 8;
   static constexpr int SmemBytes = OffMisc + 192 + 1024;
   static_assert(SmemBytes <= 232448, "shared memory budget");
@@ -77,20 +81,29 @@ struct Cfg128 {
   static constexpr uint32_t IdescPV = idesc_bf16(D, 128, 1, 1);   // A = V^T, B = P^T (MN-major)
 };
 
+// The ring's loads are numbered L = 0, 1, 2, ... (2n: K of step n, 2n + 1:
+// its V); load L goes to stage L mod 3 as that stage's m-th load, m = L / 3.
+// Since 3 is odd, a stage's loads alternate between K and V, and so do its
+// readers. Each stage therefore has a pair of full and a pair of empty
+// barriers, one per kind: every barrier then has a single waiter that sees
+// each of its phases in order (the K producer waits on EMPTY_V, the V
+// producer on EMPTY_K, the S issuer on FULL_K, the PV issuer on FULL_V), and
+// a load's phase on its own barriers is m / 2, parity (m >> 1) & 1.
 enum {
   B_ITEM_FULL = 0,   // [2] slots
   B_ITEM_EMPTY = 2,  // [2]
   B_Q_FULL = 4,
   B_Q_EMPTY = 5,     // the item's last S^T has completed
-  B_K_FULL = 6,      // [2]
-  B_V_FULL = 8,      // [2]
-  B_V_EMPTY = 10,    // [2] the PV that read the stage has completed
-  B_S_FULL = 12,     // [2] S^T buffer n & 1 written (also frees K stage n & 1)
-  B_S_FREE = 14,     // [2] both warpgroups have read S^T buffer n & 1
-  B_P_FULL = 16,     // P^T of the step written (256 arrivals)
-  B_P_EMPTY = 17,    // the PV that read P^T has completed
-  B_O_DONE = 18,     // the item's last PV has completed
-  B_O_FREE = 19      // the epilogue has read O^T (256 arrivals)
+  B_FULL_K = 6,      // [NKV] a K tile has landed in the stage
+  B_FULL_V = 9,      // [NKV] a V tile has landed in the stage
+  B_EMPTY_K = 12,    // [NKV] the S^T product that read the stage's K has completed
+  B_EMPTY_V = 15,    // [NKV] the PV product that read the stage's V has completed
+  B_S_FULL = 18,     // [2] S^T buffer n & 1 written
+  B_S_FREE = 20,     // [2] both warpgroups have read S^T buffer n & 1
+  B_P_FULL = 22,     // [2] P^T tile n & 1 written (256 arrivals)
+  B_P_EMPTY = 24,    // [2] the PV that read P^T tile n & 1 has completed
+  B_O_DONE = 26,     // the item's last PV has completed
+  B_O_FREE = 27      // the epilogue has read O^T (256 arrivals)
 };
 
 struct Item128 {
@@ -143,7 +156,7 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + C::OffMisc);
   volatile uint32_t* sTotal = reinterpret_cast<volatile uint32_t*>(smem + C::OffMisc + 8);
   volatile uint32_t* sKMeta = reinterpret_cast<volatile uint32_t*>(smem + C::OffMisc + 16);  // [2]
-  volatile uint32_t* sPMeta = reinterpret_cast<volatile uint32_t*>(smem + C::OffMisc + 24);
+  volatile uint32_t* sPMeta = reinterpret_cast<volatile uint32_t*>(smem + C::OffMisc + 24);  // [2]
   Item128* sItem = reinterpret_cast<Item128*>(smem + C::OffMisc + 32);  // [2] slots
   volatile CtaFlags* sFlags = reinterpret_cast<volatile CtaFlags*>(smem + C::OffMisc + 176);
   volatile int* sAbort = &sFlags->abort;
@@ -156,16 +169,19 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     for (int u = 0; u < 2; ++u) {
       mbar_init(bar(B_ITEM_FULL + u), 1);
       mbar_init(bar(B_ITEM_EMPTY + u), 3);  // V producer + both warpgroups
-      mbar_init(bar(B_K_FULL + u), 1);
-      mbar_init(bar(B_V_FULL + u), 1);
-      mbar_init(bar(B_V_EMPTY + u), 1);
+      mbar_init(bar(B_P_FULL + u), 256);
+      mbar_init(bar(B_P_EMPTY + u), 1);
       mbar_init(bar(B_S_FULL + u), 1);
       mbar_init(bar(B_S_FREE + u), 256);
     }
     mbar_init(bar(B_Q_FULL), 1);
     mbar_init(bar(B_Q_EMPTY), 1);
-    mbar_init(bar(B_P_FULL), 256);
-    mbar_init(bar(B_P_EMPTY), 1);
+    for (int u = 0; u < C::NKV; ++u) {
+      mbar_init(bar(B_FULL_K + u), 1);
+      mbar_init(bar(B_FULL_V + u), 1);
+      mbar_init(bar(B_EMPTY_K + u), 1);
+      mbar_init(bar(B_EMPTY_V + u), 1);
+    }
     mbar_init(bar(B_O_DONE), 1);
     mbar_init(bar(B_O_FREE), 256);
     sFlags->abort = 0;
@@ -190,7 +206,7 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     // ------------------------------------------------------------------ K producer
     int16_t* const lists = reinterpret_cast<int16_t*>(smem + C::OffList);
     uint32_t n = 0;         // walk step (one kept block per step)
-    uint32_t lastK = 0;     // bit u: stage u has an issued load; bit 2+u: its parity
+    uint32_t lastK = 0;     // bit u: stage u has had a K load; bit 8 + u: its phase parity
     uint32_t nq = 0;        // Q tiles loaded
     bool ok = true;
     for (int t = 0;; ++t) {
@@ -250,18 +266,19 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         }
         const int kvr = (int)(((size_t)b * a.Hkv + h / a.group) * a.N);
         for (int c = 0; c < cntv && ok; ++c, ++n) {
-          const uint32_t ks = n & 1;
-          // the stage's previous tile was read by the S^T of step n - 2
-          if (n >= 2) ok = ok && mbar_wait(bar(B_S_FULL + ks), ((n - 2) >> 1) & 1, wc, 3);
+          // load L = 2n into stage L mod 3 once the V that was the stage's
+          // previous load (L - 3) has been read
+          const uint32_t L = 2 * n, ks = L % C::NKV, m = L / C::NKV;
+          if (m > 0) ok = ok && mbar_wait(bar(B_EMPTY_V + ks), ((m - 1) >> 1) & 1, wc, 3);
           if (!ok) break;
-          sKMeta[ks] = step_meta(0, c == 0, c == cntv - 1, 1);
-          mbar_expect_tx(bar(B_K_FULL + ks), C::TileBytes);
+          sKMeta[n & 1] = step_meta(0, c == 0, c == cntv - 1, 1);
+          mbar_expect_tx(bar(B_FULL_K + ks), C::TileBytes);
           const int row = kvr + my_list[c] * kBS;
 #pragma unroll
           for (int hh = 0; hh < C::DH; ++hh)
-            tma_load_2d(sbase + C::OffK + ks * C::TileBytes + hh * C::Atom, &tmK, 64 * hh, row,
-                        bar(B_K_FULL + ks));
-          lastK = (lastK & ~(5u << ks)) | (1u << ks) | (((n >> 1) & 1u) << (2 + ks));
+            tma_load_2d(sbase + C::OffKV + ks * C::TileBytes + hh * C::Atom, &tmK, 64 * hh, row,
+                        bar(B_FULL_K + ks));
+          lastK = (lastK & ~(0x101u << ks)) | (1u << ks) | (((m >> 1) & 1u) << (8 + ks));
         }
       }
       n = __shfl_sync(0xffffffffu, n, 0);
@@ -270,8 +287,8 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     if (lane == 0) {
       *sTotal = n;
       // drain: every issued load has landed before the CTA may exit
-      for (int u = 0; u < 2; ++u)
-        if (lastK & (1u << u)) mbar_drain(bar(B_K_FULL + u), (lastK >> (2 + u)) & 1u, a.hdr, kKernAttnTc, 5);
+      for (int u = 0; u < C::NKV; ++u)
+        if (lastK & (1u << u)) mbar_drain(bar(B_FULL_K + u), (lastK >> (8 + u)) & 1u, a.hdr, kKernAttnTc, 5);
       if (nq > 0) mbar_drain(bar(B_Q_FULL), (nq - 1) & 1, a.hdr, kKernAttnTc, 5);
     }
   } else if (warp == 3) {
@@ -279,7 +296,7 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const int16_t* const lists = reinterpret_cast<const int16_t*>(smem + C::OffList);
     if (lane == 0) {
       uint32_t n = 0;
-      uint32_t lastV = 0;
+      uint32_t lastV = 0;   // as lastK of the K producer
       bool ok = true;
       for (int t = 0;; ++t) {
         const int slot = t & 1;
@@ -289,23 +306,24 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         if (cntv < 0) break;
         const int kvr = (int)(((size_t)it.b * a.Hkv + it.h / a.group) * a.N);
         for (int c = 0; c < cntv && ok; ++c, ++n) {
-          const uint32_t vs = n & 1;
-          // the stage's previous tile was read by the PV of step n - 2
-          if (n >= 2) ok = ok && mbar_wait(bar(B_V_EMPTY + vs), ((n - 2) >> 1) & 1, wc, 4);
+          // load L = 2n + 1 into stage L mod 3 once the K that was the
+          // stage's previous load has been read
+          const uint32_t L = 2 * n + 1, vs = L % C::NKV, m = L / C::NKV;
+          if (m > 0) ok = ok && mbar_wait(bar(B_EMPTY_K + vs), ((m - 1) >> 1) & 1, wc, 4);
           if (!ok) break;
-          mbar_expect_tx(bar(B_V_FULL + vs), C::TileBytes);
+          mbar_expect_tx(bar(B_FULL_V + vs), C::TileBytes);
           const int row = kvr + lists[slot * kMaxBlocks + c] * kBS;
 #pragma unroll
           for (int hh = 0; hh < C::DH; ++hh)
-            tma_load_2d(sbase + C::OffV + vs * C::TileBytes + hh * C::Atom, &tmV, 64 * hh, row,
-                        bar(B_V_FULL + vs));
-          lastV = (lastV & ~(5u << vs)) | (1u << vs) | (((n >> 1) & 1u) << (2 + vs));
+            tma_load_2d(sbase + C::OffKV + vs * C::TileBytes + hh * C::Atom, &tmV, 64 * hh, row,
+                        bar(B_FULL_V + vs));
+          lastV = (lastV & ~(0x101u << vs)) | (1u << vs) | (((m >> 1) & 1u) << (8 + vs));
         }
         mbar_arrive(bar(B_ITEM_EMPTY + slot));  // the slot's list has been read
         if (!ok) break;
       }
-      for (int u = 0; u < 2; ++u)
-        if (lastV & (1u << u)) mbar_drain(bar(B_V_FULL + u), (lastV >> (2 + u)) & 1u, a.hdr, kKernAttnTc, 5);
+      for (int u = 0; u < C::NKV; ++u)
+        if (lastV & (1u << u)) mbar_drain(bar(B_FULL_V + u), (lastV >> (8 + u)) & 1u, a.hdr, kKernAttnTc, 5);
     }
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------------ MMA issuers
@@ -314,15 +332,16 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       bool ok = true;
       uint32_t nq = 0;   // S issuer: items started (Q tiles consumed)
       uint32_t no = 0;   // PV issuer: items finished (O^T accumulations completed)
-      const uint64_t dK0 = smem_desc(sbase + C::OffK, 16, 1024);
+      const uint64_t dK0 = smem_desc(sbase + C::OffKV, 16, 1024);
       const uint64_t dQ0 = smem_desc(sbase + C::OffQ, 16, 1024);
-      const uint64_t dV0 = smem_desc(sbase + C::OffV, C::Atom, 1024);
+      const uint64_t dV0 = smem_desc(sbase + C::OffKV, C::Atom, 1024);
       const uint64_t dP0 = smem_desc(sbase + C::OffP, C::PBytes / 2, 1024);
       uint32_t n = 0;
       for (;; ++n) {
         const uint32_t u = n & 1;
         if (is_s) {
-          const int w = step_wait(bar(B_K_FULL + u), (n >> 1) & 1, sTotal, n, wc, 14);
+          const uint32_t L = 2 * n, ks = L % C::NKV;
+          const int w = step_wait(bar(B_FULL_K + ks), ((L / C::NKV) >> 1) & 1, sTotal, n, wc, 14);
           if (w <= 0) break;
           const uint32_t meta = sKMeta[u];
           if (meta & 2u) ok = ok && mbar_wait(bar(B_Q_FULL), nq++ & 1, wc, 13);
@@ -330,7 +349,7 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           if (n >= 2) ok = ok && mbar_wait(bar(B_S_FREE + u), ((n - 2) >> 1) & 1, wc, 15);
           tc_fence_after();
           if (ok) {
-            const uint64_t dk = dK0 + (uint64_t)((u * C::TileBytes) >> 4);
+            const uint64_t dk = dK0 + (uint64_t)((ks * C::TileBytes) >> 4);
             const uint32_t d = tmem + u * 128;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
@@ -338,26 +357,29 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                      dQ0 + (uint64_t)(((kk >> 2) * C::Atom + (kk & 3) * 32) >> 4), C::IdescS,
                      kk > 0 ? 1u : 0u);
           }
-          tc_commit(bar(B_S_FULL + u));  // also frees K stage u
+          tc_commit(bar(B_S_FULL + u));
+          tc_commit(bar(B_EMPTY_K + ks));  // the K tile's stage may be refilled
           if (meta & 4u) tc_commit(bar(B_Q_EMPTY));
         } else {
-          const int w = step_wait(bar(B_P_FULL), n & 1, sTotal, n, wc, 10);
+          const int w = step_wait(bar(B_P_FULL + u), (n >> 1) & 1, sTotal, n, wc, 10);
           if (w <= 0) break;
-          const uint32_t meta = *sPMeta;
-          ok = ok && mbar_wait(bar(B_V_FULL + u), (n >> 1) & 1, wc, 11);
+          const uint32_t meta = sPMeta[u];
+          const uint32_t L = 2 * n + 1, vs = L % C::NKV;
+          ok = ok && mbar_wait(bar(B_FULL_V + vs), ((L / C::NKV) >> 1) & 1, wc, 11);
           // a new item overwrites O^T: the previous item's epilogue has read it
           if ((meta & 2u) && no > 0) ok = ok && mbar_wait(bar(B_O_FREE), (no - 1) & 1, wc, 12);
           tc_fence_after();
           if (ok) {
-            const uint64_t dv = dV0 + (uint64_t)((u * C::TileBytes) >> 4);
+            const uint64_t dv = dV0 + (uint64_t)((vs * C::TileBytes) >> 4);
+            const uint64_t dp = dP0 + (uint64_t)((u * C::PBytes) >> 4);
             const uint32_t d = tmem + C::ColO;
 #pragma unroll
             for (int kk = 0; kk < kBS / 16; ++kk)
-              tc_mma(d, dv + (uint64_t)(kk * 128), dP0 + (uint64_t)(kk * 128), C::IdescPV,
+              tc_mma(d, dv + (uint64_t)(kk * 128), dp + (uint64_t)(kk * 128), C::IdescPV,
                      (kk > 0 || !(meta & 2u)) ? 1u : 0u);
           }
-          tc_commit(bar(B_P_EMPTY));     // P^T may be rewritten
-          tc_commit(bar(B_V_EMPTY + u)); // V stage u may be refilled
+          tc_commit(bar(B_P_EMPTY + u));    // P^T tile u may be rewritten
+          tc_commit(bar(B_EMPTY_V + vs));  // the V tile's stage may be refilled
           if (meta & 4u) {
             tc_commit(bar(B_O_DONE));
             ++no;
@@ -367,7 +389,7 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       // the tensor core has finished every MMA before TMEM is released
       if (n > 0) {
         if (is_s) mbar_drain(bar(B_S_FULL + ((n - 1) & 1)), ((n - 1) >> 1) & 1, a.hdr, kKernAttnTc, 17);
-        else mbar_drain(bar(B_P_EMPTY), (n - 1) & 1, a.hdr, kKernAttnTc, 16);
+        else mbar_drain(bar(B_P_EMPTY + ((n - 1) & 1)), ((n - 1) >> 1) & 1, a.hdr, kKernAttnTc, 16);
       }
     }
   } else {
@@ -384,7 +406,7 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     float* const sNM = reinterpret_cast<float*>(smem + C::OffM) + wg * 64;
     float* const sL = reinterpret_cast<float*>(smem + C::OffL) + wg * 64;
     float* const sA = reinterpret_cast<float*>(smem + C::OffA) + wg * 64;
-    uint8_t* const prow = smem + C::OffP + wg * (C::PBytes / 2) + r * 128;
+    uint8_t* const prow0 = smem + C::OffP + wg * (C::PBytes / 2) + r * 128;  // tile 0
     const uint32_t o_addr = tmem + lane_addr + C::ColO + q0;
     float2 l2[32];
     float tmin = INFINITY;
@@ -468,7 +490,7 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           if (c > 0) {
             // O^T holds every earlier step's contribution (the PV of step n - 1
             // has completed) before it is rescaled
-            mbar_wait<true>(bar(B_P_EMPTY), (n - 1) & 1, wc, 20);
+            mbar_wait<true>(bar(B_P_EMPTY + ((n - 1) & 1)), ((n - 1) >> 1) & 1, wc, 20);
             tc_fence_after();
             tmem_ld(o_addr, raw);
 #pragma unroll
@@ -509,15 +531,17 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             }
           }
         }
-        if (n >= 1) mbar_wait<true>(bar(B_P_EMPTY), (n - 1) & 1, wc, 24);
+        // P^T tile n & 1 was read by the PV of step n - 2
+        if (n >= 2) mbar_wait<true>(bar(B_P_EMPTY + u), ((n - 2) >> 1) & 1, wc, 24);
+        uint8_t* const prow = prow0 + u * C::PBytes;
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc)
           *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
               make_uint4(pw[4 * cc], pw[4 * cc + 1], pw[4 * cc + 2], pw[4 * cc + 3]);
-        if (r == 0 && wg == 0) *sPMeta = step_meta(0, c == 0, c == it.n - 1, 1);
+        if (r == 0 && wg == 0) sPMeta[u] = step_meta(0, c == 0, c == it.n - 1, 1);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
-        mbar_arrive(bar(B_P_FULL));
+        mbar_arrive(bar(B_P_FULL + u));
       }
       // ---------------------------------------------------------------- epilogue
       if (it.n > 0) {
