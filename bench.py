@@ -457,6 +457,7 @@ def run_ours(args, w):
         return 0
 
     peaks, peak_kind = load_peaks()
+    uses_tc = B.dsa_attn_uses_tcgen05(att.params)  # the kernel step 4 ran
     att_avg = statistics.mean(att_ms)
     sel_avg = statistics.mean(sel_ms)
     flops = kept_flops(kept, w.block, w.d)
@@ -477,7 +478,7 @@ def run_ours(args, w):
         "config": config_dict(w),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak,
-                     "traffic": recorded_traffic(w.name) if args.attn_kernel in (0, 1) else None,
+                     "traffic": recorded_traffic(w.name) if uses_tc == 1 else None,
                      "kernel": "sparse attention (dsa_sparse_attn_fwd)",
                      "peak_kind": f"{peak_kind} bf16 dense, burst",
                      "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained",
@@ -502,7 +503,8 @@ def run_ours(args, w):
                            "the neighbouring steps' computation"},
         "gpu_launches": 3 * K,
         "clocks": clocks,
-        "attn_kernel": {0: "auto", 1: "tcgen05", 2: "mma.sync"}[args.attn_kernel],
+        "attn_kernel": {0: "auto", 1: "tcgen05", 2: "mma.sync"}[args.attn_kernel]
+                       + {1: " (tcgen05)", 0: " (mma.sync)"}.get(uses_tc, "") * (args.attn_kernel == 0),
     }
     if args.select_mode != "topk":
         line["config"]["select_mode"] = args.select_mode

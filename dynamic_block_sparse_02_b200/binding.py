@@ -55,6 +55,7 @@ class dsa_params(ctypes.Structure):
 _P = ctypes.POINTER(dsa_params)
 SIGNATURES = {
     "dsa_kmax": (_sz, [_P]),
+    "dsa_attn_uses_tcgen05": (ctypes.c_int, [_P]),
     "dsa_workspace_size": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_size_t)]),
     "dsa_workspace_init": (ctypes.c_int, [_vp, _sz, _vp]),
     "dsa_workspace_set_wait_limit": (ctypes.c_int, [_vp, _sz, ctypes.c_ulonglong, _vp]),
@@ -153,6 +154,10 @@ def _check(status: int, where: str) -> None:
 
 def dsa_kmax(p: Params) -> int:
     return int(_lib.dsa_kmax(p.ref))
+
+
+def dsa_attn_uses_tcgen05(p: Params) -> int:
+    return int(_lib.dsa_attn_uses_tcgen05(p.ref))
 
 
 def dsa_workspace_size(p: Params) -> int:

@@ -85,7 +85,11 @@ typedef enum dsa_select_mode {
                                 adapts k or the threshold per input. */
 } dsa_select_mode;
 
-/* Attention kernel choice (dsa_params.attn_kernel). */
+/* Attention kernel choice (dsa_params.attn_kernel). AUTO runs the tcgen05
+ * kernel for 64x64 and 128x128 blocks and the warp-MMA kernel for 32x32
+ * blocks, where its N = 32 score products leave the tcgen05 kernel's per-step
+ * synchronisation exposed and the warp-MMA kernel is the faster one
+ * (dsa_attn_uses_tcgen05 reports the choice). */
 typedef enum dsa_attn_kernel {
   DSA_ATTN_AUTO = 0,     /* the fastest kernel this library has for the shape */
   DSA_ATTN_TCGEN05 = 1,  /* tcgen05/TMEM tensor-core kernel with TMA tile loads */
@@ -137,6 +141,12 @@ typedef struct dsa_params {
 /* Row width W of idx: min(nb, max_h k_h + local_window + n_sink). 0 for an
  * invalid or empty problem. */
 size_t dsa_kmax(const dsa_params *p);
+
+/* Which kernel the forward attention (step 4 of dsa_forward and
+ * dsa_sparse_attn_fwd) runs for p: 1 the tcgen05 kernel, 0 the warp-MMA
+ * kernel, -1 when p is invalid or asks for DSA_ATTN_TCGEN05 on a shape that
+ * kernel does not support. No device work; safe to call without a GPU. */
+int dsa_attn_uses_tcgen05(const dsa_params *p);
 
 /* Bytes of device workspace the calls below need for this problem (*bytes is
  * set on success). The first 256 bytes are a header (device error flag, work

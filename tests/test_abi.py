@@ -27,7 +27,8 @@ def test_header_declares_expected_entry_points():
     names = declared_functions()
     for n in ("dsa_block_scores", "dsa_topk_select", "dsa_sparse_attn_fwd", "dsa_forward",
               "dsa_sparse_attn_bwd", "dsa_decode_fwd", "dsa_pool_keys",
-              "dsa_workspace_size", "dsa_kmax", "dsa_check_status", "dsa_status_string"):
+              "dsa_workspace_size", "dsa_kmax", "dsa_check_status", "dsa_status_string",
+              "dsa_attn_uses_tcgen05"):
         assert n in names
 
 
@@ -105,6 +106,16 @@ def test_invalid_params_rejected_before_any_launch(change, status):
     n = ctypes.c_size_t(0)
     assert B.raw("dsa_workspace_size")(p.ref, ctypes.byref(n)) == status
     assert B.dsa_kmax(p) == 0
+
+
+def test_attention_kernel_choice_query():
+    # answers that do not depend on the driver: the warp-MMA kernel when asked
+    # for, and for 32x32 blocks under AUTO; -1 for an invalid problem
+    assert B.dsa_attn_uses_tcgen05(B.Params(**(BASE | dict(attn_kernel=B.DSA_ATTN_MMA_SYNC)))) == 0
+    assert B.dsa_attn_uses_tcgen05(B.Params(**(BASE | dict(block=32)))) == 0
+    assert B.dsa_attn_uses_tcgen05(B.Params(**(BASE | dict(d=96)))) == -1
+    assert B.dsa_attn_uses_tcgen05(B.Params(**(BASE | dict(attn_kernel=7)))) == -1
+    assert B.raw("dsa_attn_uses_tcgen05")(None) == -1
 
 
 def test_negative_per_head_budget_rejected():

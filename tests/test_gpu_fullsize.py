@@ -140,9 +140,16 @@ def test_full_workload(name):
         o_h = out.float().cpu().numpy()
         l_h = lse.cpu().numpy()
         o_fh = out_f.float().cpu().numpy()
+        # where AUTO runs the warp-MMA kernel, the tcgen05 kernel is checked too
+        o_th = l_th = None
+        if B.dsa_attn_uses_tcgen05(att.params) == 0:
+            att_t = BlockSparseAttention.from_workload(w, k_per_head=kph, attn_kernel=B.DSA_ATTN_TCGEN05)
+            att_t.sparse_attn(q, k, v, dev_i32(idx_ref), dev_i32(cnt_ref), out, lse)
+            assert att_t.check_status() == B.DSA_OK
+            o_th, l_th = out.float().cpu().numpy(), lse.cpu().numpy()
         del q, k, v, out, lse, out_f, lse_f
         items = checked_items(w)
-        acc, acc_f = Accum(), Accum()
+        acc, acc_f, acc_t = Accum(), Accum(), Accum()
         step = 2048
         for s0 in range(0, len(items), step):
             batch = items[s0:s0 + step]
@@ -154,7 +161,12 @@ def test_full_workload(name):
                         f"{name} {(b, h, i)}")
                 if np.array_equal(idx_h[b, h, i], idx_ref[b, h, i]):
                     acc_f.add(o_fh[b, h, rows].astype(np.float64), o_r)
+                if o_th is not None:
+                    acc_t.add(o_th[b, h, rows].astype(np.float64), o_r, l_th[b, h, rows].astype(np.float64),
+                              l_r, f"{name} tcgen05 {(b, h, i)}")
     acc.check(f"{name} attention on the oracle's lists")
+    if o_th is not None:
+        acc_t.check(f"{name} tcgen05 kernel on the oracle's lists")
     acc_f.check(f"{name} dsa_forward on rows selected as the oracle")
     assert acc_f.blocks >= 0.99 * acc.blocks
 

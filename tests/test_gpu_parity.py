@@ -110,6 +110,15 @@ def tc_supported(w):
     return w.block in (32, 64, 128) and w.d in (64, 128)
 
 
+def test_auto_kernel_choice_on_the_gpu():
+    # AUTO: tcgen05 for 64x64 and 128x128 blocks, the warp-MMA kernel for 32x32
+    for block, want in ((32, 0), (64, 1), (128, 1)):
+        p = B.Params(1, 4, 2, block * 16, 128, block, k_free=2)
+        assert B.dsa_attn_uses_tcgen05(p) == want, block
+        assert B.dsa_attn_uses_tcgen05(B.Params(1, 4, 2, block * 16, 128, block, k_free=2,
+                                                attn_kernel=B.DSA_ATTN_TCGEN05)) == 1
+
+
 def test_explicit_tcgen05_kernel_or_unsupported():
     for name in SMALL:
         w, kph = spec_workload(name)
