@@ -665,11 +665,15 @@ def run_backward(args, w):
     to_t = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
     q, k, v, dout = (to_t(a).to(dev) for a in (x["q"], x["k"], x["v"], do_h))
     stream = torch.cuda.Stream(device=dev)
-    att = BlockSparseAttention.from_workload(w, device=dev, stream=stream)
+    att = BlockSparseAttention.from_workload(w, attn_kernel=args.attn_kernel, device=dev, stream=stream)
     idx, cnt = att.empty_selection()
     out = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    # the tcgen05 backward (64x64 blocks, unless the warp-MMA kernel is asked
+    # for) launches prep, colbits, pairs, dQ and dK/dV; the warp-MMA path prep,
+    # colbits, dQ and dK/dV
+    tc_bwd = w.block == 64 and args.attn_kernel != 2
     with torch.cuda.stream(stream):
         att.forward(q, k, v, out, lse, idx, cnt)  # the selection and forward the backward follows
         for _ in range(args.warmup):
@@ -720,12 +724,15 @@ def run_backward(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
         "roofline": {"bound": "tensor", "achieved": tfs, "peak": peak, "unit": "TFLOP/s", "frac": tfs / peak,
-                     "traffic": None, "kernel": "backward step (prep, colbits, dq, dkv)",
+                     "traffic": None,
+                     "kernel": "backward step (prep, colbits, pairs, dQ and dK/dV passes on tcgen05)" if tc_bwd
+                     else "backward step (prep, colbits, dQ and dK/dV on mma.sync)",
                      "peak_kind": f"{peak_kind} bf16 dense, burst", "algorithmic_flops": flops,
                      "frac_of_sustained": tfs / float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))},
         "kept_blocks": kept,
         "cpu_baseline": cpu,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": (5 if tc_bwd else 4) * args.steps,
+        "attn_kernel": {0: "auto", 1: "tcgen05", 2: "mma.sync"}[args.attn_kernel],
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
