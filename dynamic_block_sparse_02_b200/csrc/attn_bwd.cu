@@ -118,7 +118,8 @@ __global__ void __launch_bounds__(256) bwd_colbits_kernel(BwdArgs a) {
   }
   if (t >= n) return;
   const int j = a.idx[row * a.W + t];
-  if (j < 0 || j > i) {
+  // the same entries as the dQ passes use: in range and above the one before
+  if (j < 0 || j > i || (t > 0 && j <= a.idx[row * a.W + t - 1])) {
     raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnBwd, (int)row, j);
     return;
   }
@@ -160,7 +161,7 @@ __global__ void __launch_bounds__(BwdCfg<BS, D>::kThreads) bwd_dq_kernel(BwdArgs
   const size_t row_id = (size_t)bh * a.nb + i;
 
   // kept list -> shared memory, 32 entries per step by warp 0, dropping
-  // out-of-range entries (flagged)
+  // out-of-range and out-of-order entries (flagged)
   if (warp == 0) {
     int n = a.cnt[row_id];
     if (n < 0 || n > a.W) {
@@ -172,7 +173,7 @@ __global__ void __launch_bounds__(BwdCfg<BS, D>::kThreads) bwd_dq_kernel(BwdArgs
     for (int t0 = 0; t0 < n; t0 += 32) {
       const int t = t0 + lane;
       const int j = t < n ? lst[t] : 0;
-      const bool bad = t < n && (j < 0 || j > i);
+      const bool bad = t < n && !list_entry_ok(lst, t, j, i, true);
       if (bad) raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnBwd, (int)row_id, j);
       const uint32_t keep = __ballot_sync(0xffffffffu, t < n && !bad);
       if ((keep >> lane) & 1u) sList[m + __popc(keep & ((1u << lane) - 1u))] = j;

@@ -257,7 +257,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmF1, const __grid_constant__ 
       int cntv = 0, diag_last = 0;
       long long pair_base = 0;
       if (!DKV) {
-        // the query block's kept list, out-of-range entries dropped (and flagged)
+        // the query block's kept list, out-of-range and out-of-order entries dropped (and flagged)
         const size_t row_id = ((size_t)b * a.Hq + h) * a.nb + i;
         int n_raw = a.cnt[row_id];
         if (n_raw < 0 || n_raw > a.W) {
@@ -270,7 +270,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmF1, const __grid_constant__ 
           const int t2 = base + lane;
           const bool in = t2 < n_raw;
           const int j = in ? lst[t2] : -1;
-          const bool valid = in && j >= 0 && j <= i;
+          const bool valid = list_entry_ok(lst, t2, j, i, in);
           if (in && !valid) raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnBwd, (int)row_id, j);
           const uint32_t m = __ballot_sync(0xffffffffu, valid);
           if (valid) my_list[cntv + __popc(m & ((1u << lane) - 1u))] = (int16_t)j;

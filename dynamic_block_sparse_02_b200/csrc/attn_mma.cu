@@ -73,7 +73,8 @@ attn_mma_kernel(AttnArgs a) {
   const int bh = b * a.Hq + h;
   const size_t row_id = (size_t)bh * a.nb + i;
 
-  // Kept list -> shared memory, dropping out-of-range entries (flagged).
+  // Kept list -> shared memory, dropping out-of-range and out-of-order
+  // entries (flagged): an entry must exceed the one before it.
   if (tid == 0) {
     int n = a.cnt[row_id];
     if (n < 0 || n > a.W) {
@@ -81,10 +82,12 @@ attn_mma_kernel(AttnArgs a) {
       n = n < 0 ? 0 : a.W;
     }
     const int32_t* lst = a.idx + row_id * a.W;
-    int m = 0;
+    int m = 0, prev = -1;
     for (int t = 0; t < n; ++t) {
       const int j = lst[t];
-      if (j < 0 || j > i) {
+      const bool ok = j >= 0 && j <= i && (t == 0 || j > prev);
+      prev = j;
+      if (!ok) {
         raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnMma, (int)row_id, j);
         continue;
       }

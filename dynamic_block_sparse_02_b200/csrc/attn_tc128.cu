@@ -237,7 +237,7 @@ attn_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         const int t2 = base + lane;
         const bool in = t2 < n_raw;
         const int j = in ? lst[t2] : -1;
-        const bool valid = in && j >= 0 && j <= i;
+        const bool valid = list_entry_ok(lst, t2, j, i, in);
         if (in && !valid) raise_error(a.hdr, DSA_ERR_DEVICE_BOUNDS, kKernAttnTc, (int)row_id, j);
         const uint32_t m = __ballot_sync(0xffffffffu, valid);
         if (valid) my_list[cntv + __popc(m & ((1u << lane) - 1u))] = (int16_t)j;

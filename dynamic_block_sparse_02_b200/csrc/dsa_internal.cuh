@@ -54,6 +54,15 @@ __device__ __forceinline__ void raise_error(WsHeader* hdr, int status, int kerne
   }
 }
 
+// Entry t = j of a caller's kept list lst (in: t < the row's count): it is
+// used only if 0 <= j <= i and j is greater than the entry before it in the
+// list (rows are ascending without repeats); other entries are skipped and
+// flagged by the caller. The entry before is read again from the list (the
+// same cache line, no state carried between entries).
+__device__ __forceinline__ bool list_entry_ok(const int32_t* lst, int t, int j, int i, bool in) {
+  return in && j >= 0 && j <= i && (t == 0 || j > lst[t - 1]);
+}
+
 // Launchers (return cudaSuccess or the launch error).
 cudaError_t launch_pool(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, float* qp,
                         float* kp, cudaStream_t st);

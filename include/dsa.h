@@ -229,8 +229,9 @@ dsa_status dsa_select_blocks_static(const dsa_params *p, const dsa_bf16 *q, cons
 /*
  * Step 4 on a caller selection. idx/cnt as above, W = dsa_kmax(p); every
  * entry n < cnt must satisfy 0 <= idx <= i, and a row must be ascending
- * without repeats (the kernel skips an out-of-range entry and sets
- * DSA_ERR_DEVICE_BOUNDS; order and repeats are not checked). out: bf16
+ * without repeats. The kernel skips, and flags with DSA_ERR_DEVICE_BOUNDS, an
+ * entry out of range or not greater than the entry before it in the row (a
+ * repeat or a step down), and attends over the rest. out: bf16
  * [B,Hq,N,d] (round to nearest even). lse: optional fp32 [B,Hq,N], natural-log
  * log-sum-exp of the scaled logits of each row. A row with no visible key
  * gets out = 0 and lse = -inf.

@@ -55,6 +55,32 @@ def gpu_backward(w, x, do_bits, idx, cnt, kernel=B.DSA_ATTN_AUTO):
     return dq, dk, dv
 
 
+def test_backward_skips_repeated_and_descending_entries():
+    # the rule of the forward: an entry not greater than the one before it is
+    # skipped and flagged; the gradients are those of the remaining lists
+    from test_gpu_parity import cleaned_lists, disorder
+    w = Workload("bad-order-bwd", 1, 4, 2, 64 * 8, 128, 64, k_free=3, local_window=1, n_sink=0)
+    x = W.make_inputs(w, seed=12)
+    idx, cnt = oracle_lists(w, x)
+    bad = disorder(idx, cnt)
+    clean, ccnt = cleaned_lists(bad, cnt, w.nb)
+    do_bits = W.f32_to_bf16_bits(np.random.default_rng(13).standard_normal(x["q"].shape).astype(np.float32))
+    rq, rk, rv = oracle.sparse_attention_backward(x["q"], x["k"], x["v"], do_bits, clean, ccnt, w.block)
+    q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+    for kern in KERNELS:
+        att = BlockSparseAttention.from_workload(w, attn_kernel=kern)
+        out = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+        att.sparse_attn(q, k, v, dev_i32(bad), dev_i32(cnt), out, lse)
+        assert att.check_status() == B.DSA_ERR_DEVICE_BOUNDS
+        dq, dk, dv = att.sparse_attn_backward(q, k, v, out, lse, dev_bf16(do_bits), dev_i32(bad), dev_i32(cnt))
+        torch.cuda.synchronize()
+        assert att.check_status() == B.DSA_ERR_DEVICE_BOUNDS
+        assert att.check_status() == B.DSA_OK
+        for name, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+            check_grad(f"{name} kernel {kern}", g.float().cpu().numpy(), r)
+
+
 def check_grad(name, g, r):
     g = np.asarray(g, dtype=np.float64)
     r = np.asarray(r, dtype=np.float64)

@@ -192,6 +192,49 @@ def test_out_of_range_index_is_skipped_and_flagged(d):
         assert_attention_close(o[0, 1, :5 * 64], o_ref[0, 1, :5 * 64], "untouched rows")
 
 
+def cleaned_lists(idx, cnt, nb):
+    """The lists the kernels use: entry t of row (b, h, i) is kept only if
+    0 <= j <= i and j is greater than entry t - 1 of the row as given."""
+    out = np.full_like(idx, -1)
+    c = np.zeros_like(cnt)
+    for (b, h, i), n in np.ndenumerate(cnt):
+        row = idx[b, h, i, :n]
+        keep = [int(j) for t, j in enumerate(row) if 0 <= j <= i and (t == 0 or j > row[t - 1])]
+        out[b, h, i, :len(keep)] = keep
+        c[b, h, i] = len(keep)
+    return out, c
+
+
+def disorder(idx_ref, cnt_ref):
+    """A repeated entry in one row and a step down in another."""
+    bad = idx_ref.copy()
+    rows = [(b, h, i) for (b, h, i), n in np.ndenumerate(cnt_ref) if n >= 3]
+    (b0, h0, i0), (b1, h1, i1) = rows[-1], rows[-2]
+    bad[b0, h0, i0, 1] = bad[b0, h0, i0, 0]                                   # repeat
+    bad[b1, h1, i1, 0], bad[b1, h1, i1, 1] = bad[b1, h1, i1, 1], bad[b1, h1, i1, 0]  # step down
+    return bad
+
+
+@pytest.mark.parametrize("d,block", [(128, 64), (64, 32), (128, 128)])
+def test_repeated_or_descending_entries_are_skipped_and_flagged(d, block):
+    w = Workload("bad-order", 1, 2, 2, block * 8, d, block, k_free=3, local_window=1, n_sink=0)
+    x = W.make_inputs(w, seed=11)
+    s64, idx_ref, cnt_ref = oracle_reference(w, x, None)
+    bad = disorder(idx_ref, cnt_ref)
+    clean, ccnt = cleaned_lists(bad, cnt_ref, w.nb)
+    assert not np.array_equal(clean, idx_ref)
+    o_ref, l_ref = oracle.sparse_attention(x["q"], x["k"], x["v"], clean, ccnt, w.block)
+    q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+    for kern in (B.DSA_ATTN_AUTO, B.DSA_ATTN_TCGEN05, B.DSA_ATTN_MMA_SYNC):
+        a2 = BlockSparseAttention.from_workload(w, attn_kernel=kern)
+        out, lse = a2.empty_out(), a2.empty_lse()
+        a2.sparse_attn(q, k, v, dev_i32(bad), dev_i32(cnt_ref), out, lse)
+        assert a2.check_status() == B.DSA_ERR_DEVICE_BOUNDS, kern
+        assert a2.check_status() == B.DSA_OK
+        assert_attention_close(out.double().cpu().numpy(), o_ref, f"kernel {kern}")
+        assert_lse_close(lse.double().cpu().numpy(), l_ref, f"kernel {kern}")
+
+
 def test_cuda_graph_capture_replays_forward():
     w = WORKLOADS["tiny"]
     x = W.make_inputs(w)
