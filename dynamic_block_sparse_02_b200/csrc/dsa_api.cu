@@ -291,9 +291,7 @@ int dsa_attn_uses_tcgen05(const dsa_params* p) {
     case DSA_ATTN_TCGEN05: return tc_ok ? 1 : -1;
     case DSA_ATTN_MMA_SYNC: return 0;
     default:
-      // 32x32 blocks: the warp-MMA kernel is faster (4 x 16 heads x 16384 rows,
-      // d = 64: 1.13 ms against 1.76 ms per attention launch)
-      return tc_ok && s.bs != 32 ? 1 : 0;
+      return tc_ok ? 1 : 0;
   }
 }
 

@@ -86,10 +86,8 @@ typedef enum dsa_select_mode {
 } dsa_select_mode;
 
 /* Attention kernel choice (dsa_params.attn_kernel). AUTO runs the tcgen05
- * kernel for 64x64 and 128x128 blocks and the warp-MMA kernel for 32x32
- * blocks, where its N = 32 score products leave the tcgen05 kernel's per-step
- * synchronisation exposed and the warp-MMA kernel is the faster one
- * (dsa_attn_uses_tcgen05 reports the choice). */
+ * kernel for every supported shape (block 32, 64 or 128, d 64 or 128) and the
+ * warp-MMA kernel otherwise; dsa_attn_uses_tcgen05 reports the choice. */
 typedef enum dsa_attn_kernel {
   DSA_ATTN_AUTO = 0,     /* the fastest kernel this library has for the shape */
   DSA_ATTN_TCGEN05 = 1,  /* tcgen05/TMEM tensor-core kernel with TMA tile loads */

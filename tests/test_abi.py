@@ -110,9 +110,8 @@ def test_invalid_params_rejected_before_any_launch(change, status):
 
 def test_attention_kernel_choice_query():
     # answers that do not depend on the driver: the warp-MMA kernel when asked
-    # for, and for 32x32 blocks under AUTO; -1 for an invalid problem
+    # for, -1 for an invalid problem
     assert B.dsa_attn_uses_tcgen05(B.Params(**(BASE | dict(attn_kernel=B.DSA_ATTN_MMA_SYNC)))) == 0
-    assert B.dsa_attn_uses_tcgen05(B.Params(**(BASE | dict(block=32)))) == 0
     assert B.dsa_attn_uses_tcgen05(B.Params(**(BASE | dict(d=96)))) == -1
     assert B.dsa_attn_uses_tcgen05(B.Params(**(BASE | dict(attn_kernel=7)))) == -1
     assert B.raw("dsa_attn_uses_tcgen05")(None) == -1

@@ -111,8 +111,8 @@ def tc_supported(w):
 
 
 def test_auto_kernel_choice_on_the_gpu():
-    # AUTO: tcgen05 for 64x64 and 128x128 blocks, the warp-MMA kernel for 32x32
-    for block, want in ((32, 0), (64, 1), (128, 1)):
+    # AUTO: the tcgen05 kernels for every block size
+    for block, want in ((32, 1), (64, 1), (128, 1)):
         p = B.Params(1, 4, 2, block * 16, 128, block, k_free=2)
         assert B.dsa_attn_uses_tcgen05(p) == want, block
         assert B.dsa_attn_uses_tcgen05(B.Params(1, 4, 2, block * 16, 128, block, k_free=2,
