@@ -17,7 +17,13 @@ import oracle
 TIE_REL = 1e-5
 ATOL_MAX = 2e-2
 REL_RMS = 5e-3
-LSE_ATOL = 2e-3
+# Log-sum-exp of a row, natural log: the row sum adds the bf16-rounded P (each
+# within 2^-8 of its fp32 value, the bf16 unit roundoff), so ln(row sum) is
+# within -ln(1 - 2^-8) = 3.92e-3; the fp32 sums add at most n * 2^-24 relative
+# (2.6e-4 at the 4,288 keys of a 32K row) and the fp32 logits and ex2.approx
+# about 1e-5. A sharp softmax, where one P carries the sum, reaches the first
+# term; many comparable terms average it out.
+LSE_ATOL = 4.5e-3
 
 
 def dev_bf16(bits: np.ndarray) -> torch.Tensor:

@@ -55,6 +55,20 @@ def gpu_backward(w, x, do_bits, idx, cnt, kernel=B.DSA_ATTN_AUTO):
     return dq, dk, dv
 
 
+@pytest.mark.parametrize("scale", [0.4, 0.03])
+def test_backward_custom_scale(scale):
+    w = Workload("scale-bwd", 1, 4, 2, 64 * 10, 128, 64, k_free=3, local_window=1, n_sink=1, scale=scale)
+    x = W.make_inputs(w, seed=14)
+    idx, cnt = oracle_lists(w, x)
+    do_bits = W.f32_to_bf16_bits(np.random.default_rng(15).standard_normal(x["q"].shape).astype(np.float32))
+    rq, rk, rv = oracle.sparse_attention_backward(x["q"], x["k"], x["v"], do_bits, idx, cnt, w.block,
+                                                  scale=scale)
+    for kern in KERNELS:
+        dq, dk, dv = gpu_backward(w, x, do_bits, idx, cnt, kern)
+        for name, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+            check_grad(f"{name} kernel {kern} scale {scale}", g.float().cpu().numpy(), r)
+
+
 def test_backward_skips_repeated_and_descending_entries():
     # the rule of the forward: an entry not greater than the one before it is
     # skipped and flagged; the gradients are those of the remaining lists

@@ -61,7 +61,7 @@ def run_decode(w, x, L, mode, tau=0.0, qscale=1.0):
     torch.cuda.synchronize()
     assert att.check_status() == B.DSA_OK
     ref = oracle.decode(qtok, x["k"], x["v"], L, bs, w.k_free, w.local_window, w.n_sink,
-                        mode=mode, tau=tau, return_scores=True)
+                        scale=w.scale, mode=mode, tau=tau, return_scores=True)
     return att, kp, (idx.cpu().numpy(), cnt.cpu().numpy(), out.double().cpu().numpy(),
                      lse.cpu().numpy().astype(np.float64)), ref
 
@@ -70,7 +70,7 @@ def check(w, L, got, ref, tau=None):
     idx_g, cnt_g, out_g, lse_g = got
     idx_r, cnt_r, out_r, lse_r, s64 = ref
     i = (L - 1) // w.block
-    scale = 1.0 / np.sqrt(w.d)
+    scale = w.scale if w.scale else 1.0 / np.sqrt(w.d)
     same = np.zeros((w.B, w.Hq), dtype=bool)
     for b in range(w.B):
         for h in range(w.Hq):
@@ -112,6 +112,17 @@ def test_decode_parity(name, mode):
     kp_ref = oracle.pool_blocks(x["k"][:, :, :nfull * bs], bs)
     np.testing.assert_allclose(kp.cpu().numpy()[:, :, :nfull].astype(np.float64), kp_ref, rtol=1e-5,
                                atol=1e-6)
+
+
+@pytest.mark.parametrize("mode", ["topk", "group"])
+def test_decode_custom_scale(mode):
+    # a softmax scale other than 1/sqrt(d), large enough that the running
+    # maxima move by many powers of two between blocks
+    w = Workload("scale", 1, 8, 2, 64 * 24, 128, 64, k_free=5, local_window=2, n_sink=1, scale=0.45)
+    x = W.make_inputs(w, seed=53)
+    for L in (1, 64, 65, 777, 64 * 24):
+        att, kp, got, ref = run_decode(w, x, L, mode)
+        check(w, L, got, ref)
 
 
 def test_decode_threshold():

@@ -235,6 +235,25 @@ def test_repeated_or_descending_entries_are_skipped_and_flagged(d, block):
         assert_lse_close(lse.double().cpu().numpy(), l_ref, f"kernel {kern}")
 
 
+@pytest.mark.parametrize("block,d,scale", [(64, 128, 0.5), (32, 64, 0.02), (128, 128, 0.4), (64, 64, 1.0)])
+def test_custom_scale_every_kernel(block, d, scale):
+    # a softmax scale other than 1/sqrt(d): sharp ones move the running maxima
+    # by many powers of two from block to block (the rescale path), a small one
+    # flattens the weights
+    w = Workload("scale", 2, 4, 2, block * 10, d, block, k_free=3, local_window=1, n_sink=1, scale=scale)
+    x = W.make_inputs(w, seed=21)
+    s64, idx_ref, cnt_ref = oracle_reference(w, x, None)
+    o_ref, l_ref = oracle.sparse_attention(x["q"], x["k"], x["v"], idx_ref, cnt_ref, w.block, scale=scale)
+    q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+    for kern in (B.DSA_ATTN_AUTO, B.DSA_ATTN_TCGEN05, B.DSA_ATTN_MMA_SYNC):
+        a2 = BlockSparseAttention.from_workload(w, attn_kernel=kern)
+        out, lse = a2.empty_out(), a2.empty_lse()
+        a2.sparse_attn(q, k, v, dev_i32(idx_ref), dev_i32(cnt_ref), out, lse)
+        assert a2.check_status() == B.DSA_OK
+        assert_attention_close(out.double().cpu().numpy(), o_ref, f"kernel {kern} scale {scale}")
+        assert_lse_close(lse.double().cpu().numpy(), l_ref, f"kernel {kern} scale {scale}")
+
+
 def test_cuda_graph_capture_replays_forward():
     w = WORKLOADS["tiny"]
     x = W.make_inputs(w)
