@@ -254,6 +254,28 @@ def test_custom_scale_every_kernel(block, d, scale):
         assert_lse_close(lse.double().cpu().numpy(), l_ref, f"kernel {kern} scale {scale}")
 
 
+@pytest.mark.parametrize("block,d", [(64, 128), (32, 64), (128, 128)])
+def test_forward_is_deterministic(block, d):
+    # persistent CTAs take work items from a global counter, so which CTA runs
+    # which item changes from run to run; each item's sums run in a fixed
+    # order, so two runs agree bit for bit
+    w = Workload("det", 2, 8, 2, block * 48, d, block, k_free=9, local_window=2, n_sink=1)
+    x = W.make_inputs(w, seed=31)
+    q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+    for kern in (B.DSA_ATTN_AUTO, B.DSA_ATTN_MMA_SYNC):
+        att = BlockSparseAttention.from_workload(w, attn_kernel=kern)
+        runs = []
+        for _ in range(2):
+            idx, cnt = att.empty_selection()
+            out, lse = att.empty_out(), att.empty_lse()
+            att.forward(q, k, v, out, lse, idx, cnt)
+            torch.cuda.synchronize()
+            runs.append((out, lse, idx, cnt))
+        assert att.check_status() == B.DSA_OK
+        for ta, tb in zip(*runs):
+            assert torch.equal(ta, tb), kern
+
+
 def test_cuda_graph_capture_replays_forward():
     w = WORKLOADS["tiny"]
     x = W.make_inputs(w)
