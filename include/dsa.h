@@ -89,7 +89,7 @@ typedef enum dsa_select_mode {
  * kernel for every supported shape (block 32, 64 or 128, d 64 or 128) and the
  * warp-MMA kernel otherwise; dsa_attn_uses_tcgen05 reports the choice. */
 typedef enum dsa_attn_kernel {
-  DSA_ATTN_AUTO = 0,     /* the fastest kernel this library has for the shape */
+  DSA_ATTN_AUTO = 0,     /* the tcgen05 kernel where the shape has one, else warp-MMA */
   DSA_ATTN_TCGEN05 = 1,  /* tcgen05/TMEM tensor-core kernel with TMA tile loads */
   DSA_ATTN_MMA_SYNC = 2  /* warp-level mma.sync kernel (the legacy tensor-core path) */
 } dsa_attn_kernel;
